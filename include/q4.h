@@ -1,0 +1,159 @@
+/*
+ * q4.h -- C ABI of libq4: grouped symmetric round-to-nearest (RTN) int4/int8
+ * weight quantization and the quantized matmul, on one NVIDIA B200 (sm_100a).
+ *
+ * The quantization rule is the one of pack()/unpack() on the page
+ * "量化推理：INT8/INT4 的体积、困惑度与速度为什么不同步" and of "Huit bits,
+ * puis quatre", section "Arrondir":
+ *   - flatten the weight tensor row-major and cut it into groups of `group`
+ *     consecutive values;
+ *   - scale = max|w| / qmax in fp32 (qmax = 7 for int4, 127 for int8); a
+ *     scale that comes out as 0 is replaced by 1;
+ *   - code = clip(rint(w / scale), -qmax, qmax), the quotient being one IEEE
+ *     fp32 division and rint rounding half to even;
+ *   - int4: byte t of the payload = (code[2t] + 8) | (code[2t+1] + 8) << 4
+ *     (even element in the low nibble); int8: the code's two's-complement byte;
+ *   - dequantized weight w' = float(code) * scale (one fp32 multiplication).
+ *
+ * Conventions for every call:
+ *   - Matrices are row-major. A weight matrix W is [rows = N output
+ *     channels][cols = K inputs]; activations x are [M][K]; y is [M][N].
+ *   - Every pointer argument is a DEVICE pointer (cudaMalloc'd or torch
+ *     memory on the current device) owned by the caller; the library
+ *     allocates nothing, keeps no pointer after a call returns and holds no
+ *     global state.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only
+ *     enqueue work: they return before the GPU finishes. Argument errors are
+ *     detected on the host BEFORE anything is enqueued, and nothing is
+ *     enqueued when a call returns an error.
+ *   - No call falls back to the CPU: a shape a kernel does not cover returns
+ *     Q4_ERR_UNSUPPORTED.
+ */
+#ifndef Q4_H
+#define Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum q4_status {
+    Q4_OK = 0,
+    Q4_ERR_ARG = 1,         /* a null pointer, bits not 4/8, group < 1, a shape the format cannot hold */
+    Q4_ERR_UNSUPPORTED = 2, /* a valid format that this kernel does not cover (see each call) */
+    Q4_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
+    Q4_ERR_NONFINITE = 4,   /* qpack saw Inf or NaN (reported through its status word) */
+    Q4_ERR_WORKSPACE = 5    /* qgemm workspace null, too small or not 256-byte aligned */
+} q4_status;
+
+typedef enum q4_xdtype {
+    Q4_X_F32 = 0,  /* x is float32 */
+    Q4_X_BF16 = 1  /* x is bfloat16 (raw 16-bit values) */
+} q4_xdtype;
+
+/* Bits OR-ed into the optional device status words of qpack and qgemm. */
+#define Q4_STATUS_NONFINITE 1u /* qpack: a group holds Inf or NaN */
+#define Q4_STATUS_TIMEOUT 2u   /* qgemm: a bounded wait inside a kernel gave up; y is invalid */
+
+/* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
+Q4_API int q4_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+Q4_API const char *q4_status_str(q4_status s);
+
+/* Bytes of packed codes for rows*cols weights: rows*cols*bits/8 (pack()'s
+ * payload length check on the "量化推理" page). Returns 0 for invalid
+ * arguments (negative sizes, bits not 4/8, odd rows*cols with bits = 4). */
+Q4_API size_t q4_payload_bytes(int64_t rows, int64_t cols, int bits);
+
+/* Number of fp32 scales: rows*cols/group, one per group. Returns -1 when
+ * group < 1 or does not divide rows*cols. */
+Q4_API int64_t q4_num_scales(int64_t rows, int64_t cols, int64_t group);
+
+/*
+ * qpack -- quantize and pack (pack() on the "量化推理" page; the rule of
+ * "Huit bits, puis quatre", section "Arrondir").
+ *   w        [rows*cols] fp32, row-major, 16-byte alignment recommended
+ *   bits     4 or 8
+ *   group    1 <= group, group divides rows*cols; groups run over the
+ *            flattened tensor, so a group may span rows (group = rows*cols
+ *            gives one scale for the whole tensor)
+ *   payload  out, q4_payload_bytes(rows, cols, bits) bytes
+ *   scales   out, q4_num_scales(rows, cols, group) floats
+ *   status_word  optional (may be NULL) device uint32; the kernels OR
+ *            Q4_STATUS_NONFINITE into it when any weight is Inf or NaN (the
+ *            outputs are then unspecified for that group). The caller zeroes
+ *            it and reads it after synchronizing the stream.
+ * Errors: Q4_ERR_ARG (null w/payload/scales, bits, group, odd rows*cols for
+ * int4, negative sizes), Q4_ERR_CUDA. rows*cols == 0 enqueues nothing.
+ * Results are bit-identical to the definition above for every input.
+ */
+Q4_API q4_status qpack(const float *w, int64_t rows, int64_t cols, int bits, int64_t group,
+                uint8_t *payload, float *scales, uint32_t *status_word, void *stream);
+
+/*
+ * qdequant -- decode packed codes to fp32 weights (unpack() on the "量化推理"
+ * page): w_out[i] = float(code[i]) * scales[i / group], bit-exact.
+ *   payload  [q4_payload_bytes(rows, cols, bits)] bytes from qpack
+ *   scales   [q4_num_scales(rows, cols, group)] floats
+ *   w_out    out, [rows*cols] fp32
+ * Errors: as qpack. rows*cols == 0 enqueues nothing.
+ */
+Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t rows, int64_t cols,
+                   int bits, int64_t group, float *w_out, void *stream);
+
+/*
+ * Workspace bytes that qgemm needs for this problem (0 when it needs none, which
+ * is the case for every shape the decode GEMV takes). Same arguments as qgemm.
+ * Returns 0 also for arguments qgemm rejects. Depends only on the arguments, not
+ * on the device.
+ */
+Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
+                                q4_xdtype xt);
+
+/*
+ * qgemm -- y[m][n] = sum_k x[m][k] * w'[n][k], w' the dequantized weights,
+ * computed from the packed codes without materialising w' (the
+ * QuantizedMatmul of "Huit bits, puis quatre", section "Ranger des entiers
+ * dans des f32": the same numbers as the product with the dequantized
+ * weights, up to the order of the sums).
+ *   x        [M][K], fp32 or bf16 per xt, row-major, 16-byte aligned
+ *   payload  [N][K*bits/8] bytes from qpack of an [N][K] matrix, 16-byte aligned
+ *   scales   [N*K/group] floats from the same qpack
+ *   y        out, [M][N] fp32
+ *   workspace  device scratch of at least q4_qgemm_workspace_bytes(...)
+ *            bytes, 256-byte aligned, owned by the caller; may be NULL when
+ *            that size is 0. Its contents need no initialisation and are
+ *            meaningless after the call. Two calls that may run at the same
+ *            time must not share a workspace.
+ *   status_word  optional (may be NULL) device uint32. Every wait inside the
+ *            kernels is bounded; if one ever gives up, Q4_STATUS_TIMEOUT is
+ *            OR-ed into this word and y must be treated as invalid. The
+ *            caller zeroes it and reads it after synchronizing the stream.
+ * Paths: M <= 63, or fp32 x at any M: the fused unpack->dequant->GEMV kernel
+ * (rows of x in chunks of 16). bf16 x with M >= 64: the tensor-core GEMM.
+ * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
+ * finite inputs (y_exact = the fp64 sum).
+ * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0, group divides K and
+ * group % 32 == 0 (per-channel scales are group = K); for int8 group % 16
+ * == 0 suffices. M, N >= 0; M == 0 or N == 0 enqueues nothing.
+ * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
+ * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
+ */
+Q4_API q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H */

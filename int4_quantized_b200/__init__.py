@@ -1,0 +1,190 @@
+"""int4_quantized_b200 -- Python binding of libq4 (include/q4.h), B200 / sm_100a.
+
+Symmetric round-to-nearest weight quantization with one fp32 scale per group of g
+consecutive weights (pack()/unpack() of the "量化推理：INT8/INT4 ..." page; "Huit bits,
+puis quatre", section "Arrondir"), and the quantized matmul that reads the packed codes.
+
+This module only marshals arguments: it turns torch CUDA tensors into device pointers
+and the current CUDA stream into a cudaStream_t, and checks status codes. Every step of
+the computation runs in the CUDA kernels of libq4.so. There is no CPU fallback: if the
+library is missing or a call is unsupported, an exception is raised.
+
+    payload, scales = qpack(w, bits=4, group=128)           # w: [N, K] float32 CUDA tensor
+    w_deq = qdequant(payload, scales, (N, K), 4, 128)        # float32, bit-exact
+    y = qgemm(x, payload, scales, N, K, 4, 128)              # x: [M, K] fp32 or bf16 -> y [M, N]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "Q4Error", "lib", "lib_path", "payload_bytes", "num_scales", "qgemm_workspace_bytes",
+    "qpack", "qdequant", "qgemm", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
+    "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_X_F32", "Q4_X_BF16", "STATUS_NONFINITE", "STATUS_TIMEOUT",
+]
+
+Q4_OK, Q4_ERR_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_CUDA, Q4_ERR_NONFINITE, Q4_ERR_WORKSPACE = range(6)
+Q4_X_F32, Q4_X_BF16 = 0, 1
+STATUS_NONFINITE = 1
+STATUS_TIMEOUT = 2
+
+lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libq4.so")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {lib().q4_status_str(code).decode()} (status {code})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libq4.so (built in-tree by ``python -m int4_quantized_b200._build``)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(lib_path):
+                    raise ImportError(
+                        f"libq4.so is not built at {lib_path}; run `python -m int4_quantized_b200._build`")
+                L = ctypes.CDLL(lib_path)
+                i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+                L.q4_version.restype = i32
+                L.q4_status_str.argtypes = [i32]
+                L.q4_status_str.restype = ctypes.c_char_p
+                L.q4_payload_bytes.argtypes = [i64, i64, i32]
+                L.q4_payload_bytes.restype = sz
+                L.q4_num_scales.argtypes = [i64, i64, i64]
+                L.q4_num_scales.restype = i64
+                L.qpack.argtypes = [vp, i64, i64, i32, i64, vp, vp, vp, vp]
+                L.qpack.restype = i32
+                L.qdequant.argtypes = [vp, vp, i64, i64, i32, i64, vp, vp]
+                L.qdequant.restype = i32
+                L.q4_qgemm_workspace_bytes.argtypes = [i64, i64, i64, i32, i64, i32]
+                L.q4_qgemm_workspace_bytes.restype = sz
+                L.qgemm.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, sz, vp, vp]
+                L.qgemm.restype = i32
+                _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(code: int, what: str):
+    if code != Q4_OK:
+        raise Q4Error(code, what)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def payload_bytes(rows: int, cols: int, bits: int) -> int:
+    return int(lib().q4_payload_bytes(rows, cols, bits))
+
+
+def num_scales(rows: int, cols: int, group: int) -> int:
+    return int(lib().q4_num_scales(rows, cols, group))
+
+
+def qgemm_workspace_bytes(M: int, N: int, K: int, bits: int, group: int, x_dtype=torch.float32) -> int:
+    xt = Q4_X_BF16 if x_dtype == torch.bfloat16 else Q4_X_F32
+    return int(lib().q4_qgemm_workspace_bytes(M, N, K, bits, group, xt))
+
+
+def qpack(w: torch.Tensor, bits: int, group: int, payload: Optional[torch.Tensor] = None,
+          scales: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None
+          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Quantize a float32 CUDA tensor (flattened row-major) -> (payload uint8, scales float32)."""
+    _cuda(w, "w", torch.float32)
+    rows = w.shape[0] if w.dim() >= 1 else 1
+    cols = w.numel() // rows if rows else 0
+    nb = payload_bytes(rows, cols, bits)
+    ns = num_scales(rows, cols, group)
+    if payload is None:
+        payload = torch.empty(nb, dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(max(ns, 0), dtype=torch.float32, device=w.device)
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    with torch.cuda.device(w.device):
+        _check(lib().qpack(_ptr(w), rows, cols, bits, group, _ptr(payload), _ptr(scales),
+                           _ptr(status), _stream(w.device)), "qpack")
+    return payload, scales
+
+
+def qdequant(payload: torch.Tensor, scales: torch.Tensor, shape: Sequence[int], bits: int, group: int,
+             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Decode packed codes -> float32 tensor of `shape` (code * scale, bit-exact)."""
+    _cuda(payload, "payload", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    shape = tuple(int(s) for s in shape)
+    rows = shape[0] if shape else 1
+    n = 1
+    for s in shape:
+        n *= s
+    cols = n // rows if rows else 0
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=payload.device)
+    with torch.cuda.device(payload.device):
+        _check(lib().qdequant(_ptr(payload), _ptr(scales), rows, cols, bits, group, _ptr(out),
+                              _stream(payload.device)), "qdequant")
+    return out
+
+
+_ws_cache = {}
+
+
+def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
+    key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = buf
+    return buf
+
+
+def qgemm(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, N: int, K: int, bits: int,
+          group: int, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+          status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y[M, N] = x[M, K] @ W'^T from the packed codes (x float32 or bfloat16)."""
+    _cuda(x, "x")
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _cuda(payload, "payload", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    x2 = x.reshape(-1, K)
+    M = x2.shape[0]
+    xt = Q4_X_BF16 if x.dtype == torch.bfloat16 else Q4_X_F32
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _cuda(out, "out", torch.float32)
+    need = int(lib().q4_qgemm_workspace_bytes(M, N, K, bits, group, xt))
+    if workspace is None and need > 0:
+        workspace = _workspace(x.device, need)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    with torch.cuda.device(x.device):
+        _check(lib().qgemm(_ptr(x2), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group, _ptr(out),
+                           _ptr(workspace), ws_bytes, _ptr(status), _stream(x.device)), "qgemm")
+    return out

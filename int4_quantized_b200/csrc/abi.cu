@@ -1,0 +1,130 @@
+// abi.cu -- the extern "C" entry points declared in include/q4.h.
+//
+// Every call validates its arguments on the host before enqueuing anything, then
+// launches the kernels on the caller's stream. Nothing is allocated here and no state
+// survives a call.
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace {
+
+// qgemm's task split is planned for a full B200 (148 SMs) whatever device runs it, so
+// the workspace size is a pure function of the problem and needs no CUDA call.
+constexpr int kPlanSMs = 148;
+
+inline int device_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+q4_status check_format(int64_t rows, int64_t cols, int bits, int64_t group, int64_t *n) {
+    if (bits != 4 && bits != 8) return Q4_ERR_ARG;
+    if (group < 1) return Q4_ERR_ARG;
+    if (!mul_ok(rows, cols, n)) return Q4_ERR_ARG;
+    if (*n % group != 0) return Q4_ERR_ARG;
+    if (bits == 4 && (*n % 2) != 0) return Q4_ERR_ARG;
+    return Q4_OK;
+}
+
+// Path selection for qgemm: returns Q4_OK and fills the plan, or the reason it cannot run.
+q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q4_xdtype xt,
+                     q4::GemvPlan *pl) {
+    if (bits != 4 && bits != 8) return Q4_ERR_ARG;
+    if (M < 0 || N < 0 || K < 1 || group < 1) return Q4_ERR_ARG;
+    if (xt != Q4_X_F32 && xt != Q4_X_BF16) return Q4_ERR_ARG;
+    if (K % group != 0) return Q4_ERR_UNSUPPORTED;
+    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, group, kPlanSMs, pl))
+        return Q4_ERR_UNSUPPORTED;
+    return Q4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int q4_version(void) { return 100; }
+
+const char *q4_status_str(q4_status s) {
+    switch (s) {
+        case Q4_OK: return "ok";
+        case Q4_ERR_ARG: return "invalid argument";
+        case Q4_ERR_UNSUPPORTED: return "shape or format not covered by this kernel";
+        case Q4_ERR_CUDA: return "CUDA error";
+        case Q4_ERR_NONFINITE: return "non-finite weight in a group";
+        case Q4_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    }
+    return "unknown status";
+}
+
+size_t q4_payload_bytes(int64_t rows, int64_t cols, int bits) {
+    int64_t n;
+    if ((bits != 4 && bits != 8) || !mul_ok(rows, cols, &n)) return 0;
+    if (bits == 4 && n % 2) return 0;
+    return (size_t)(bits == 8 ? n : n / 2);
+}
+
+int64_t q4_num_scales(int64_t rows, int64_t cols, int64_t group) {
+    int64_t n;
+    if (group < 1 || !mul_ok(rows, cols, &n) || n % group) return -1;
+    return n / group;
+}
+
+q4_status qpack(const float *w, int64_t rows, int64_t cols, int bits, int64_t group,
+                uint8_t *payload, float *scales, uint32_t *status_word, void *stream) {
+    int64_t n;
+    q4_status st = check_format(rows, cols, bits, group, &n);
+    if (st != Q4_OK) return st;
+    if (n == 0) return Q4_OK;
+    if (!w || !payload || !scales) return Q4_ERR_ARG;
+    cudaError_t e = q4::launch_qpack(w, n, bits, group, payload, scales, status_word,
+                                     as_stream(stream), device_sms());
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+q4_status qdequant(const uint8_t *payload, const float *scales, int64_t rows, int64_t cols,
+                   int bits, int64_t group, float *w_out, void *stream) {
+    int64_t n;
+    q4_status st = check_format(rows, cols, bits, group, &n);
+    if (st != Q4_OK) return st;
+    if (n == 0) return Q4_OK;
+    if (!payload || !scales || !w_out) return Q4_ERR_ARG;
+    cudaError_t e = q4::launch_qdequant(payload, scales, n, bits, group, w_out, as_stream(stream),
+                                        device_sms());
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
+                                q4_xdtype xt) {
+    q4::GemvPlan pl;
+    if (plan_qgemm(M, N, K, bits, group, xt, &pl) != Q4_OK) return 0;
+    return pl.bytes;
+}
+
+q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream) {
+    q4::GemvPlan pl;
+    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &pl);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !payload || !scales || !y) return Q4_ERR_ARG;
+    if ((uintptr_t)payload % 16 || (uintptr_t)x % 16) return Q4_ERR_UNSUPPORTED;
+    if ((uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
+    if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return Q4_ERR_WORKSPACE;
+    cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,
+                                    status_word, as_stream(stream));
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+}  // extern "C"

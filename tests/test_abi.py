@@ -1,0 +1,109 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, sizes
+buffers, and rejects bad arguments on the host before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from int4_quantized_b200 import _build
+
+    _build.build()
+    import int4_quantized_b200 as m
+
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "q4.h")).read()
+    return re.findall(r"^Q4_API\s[^;(]*?\b(\w+)\s*\(", src, re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"qpack", "qdequant", "qgemm", "q4_payload_bytes", "q4_num_scales",
+            "q4_qgemm_workspace_bytes", "q4_status_str", "q4_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(q4):
+    lib = q4.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_sizes(q4):
+    assert q4.payload_bytes(4096, 4096, 4) == 4096 * 4096 // 2
+    assert q4.payload_bytes(4096, 4096, 8) == 4096 * 4096
+    assert q4.payload_bytes(3, 3, 4) == 0          # odd count cannot be nibble-paired
+    assert q4.payload_bytes(-1, 3, 8) == 0
+    assert q4.payload_bytes(1, 8, 5) == 0
+    assert q4.num_scales(11008, 4096, 128) == 11008 * 32
+    assert q4.num_scales(2, 3, 4) == -1
+    assert q4.num_scales(2, 3, 0) == -1
+    assert q4.lib().q4_version() >= 100
+
+
+def test_status_strings(q4):
+    for code in range(6):
+        assert q4.lib().q4_status_str(code)
+    assert q4.lib().q4_status_str(99) == b"unknown status"
+
+
+FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("rows,cols,bits,group,ptr_ok,expect", [
+    (4, 32, 3, 32, True, 1),        # bits
+    (4, 32, 4, 0, True, 1),         # group
+    (4, 32, 4, 48, True, 1),        # group does not divide n
+    (1, 3, 4, 3, True, 1),          # odd n for int4
+    (-1, 32, 8, 32, True, 1),       # negative size
+    (4, 32, 8, 32, False, 1),       # null pointers
+    (0, 32, 8, 32, False, 0),       # empty: nothing to do, no pointer needed
+])
+def test_qpack_validation(q4, rows, cols, bits, group, ptr_ok, expect):
+    p = FAKE if ptr_ok else None
+    assert q4.lib().qpack(p, rows, cols, bits, group, p, p, None, None) == expect
+    assert q4.lib().qdequant(p, p, rows, cols, bits, group, p, None) == expect
+
+
+@pytest.mark.parametrize("M,N,K,bits,group,xt,expect", [
+    (1, 64, 128, 3, 128, 0, 1),     # bits
+    (1, 64, 128, 4, 0, 0, 1),       # group
+    (1, 64, 128, 4, 128, 7, 1),     # x dtype
+    (1, 64, 96, 4, 64, 0, 2),       # group does not divide K
+    (1, 64, 48, 4, 48, 0, 2),       # K % 32
+    (1, 64, 128, 4, 16, 0, 2),      # int4 group % 32
+    (1, 64, 128, 8, 8, 0, 2),       # int8 group % 16
+    (-1, 64, 128, 4, 128, 0, 1),    # negative M
+])
+def test_qgemm_validation(q4, M, N, K, bits, group, xt, expect):
+    assert q4.lib().qgemm(FAKE, xt, M, FAKE, FAKE, N, K, bits, group, FAKE, FAKE, 1 << 30, None, None) == expect
+
+
+def test_qgemm_workspace_rules(q4):
+    lib = q4.lib()
+    # the decode GEMV needs no global scratch at all
+    for M in (1, 8, 16, 40):
+        assert lib.q4_qgemm_workspace_bytes(M, 4096, 4096, 4, 128, 0) == 0
+    # a workspace that is given must be 256-byte aligned
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ctypes.c_void_p(0x100010), 1 << 20, None, None) == 5
+    # misaligned payload / x are reported before anything is enqueued
+    assert lib.qgemm(FAKE, 0, 8, ctypes.c_void_p(0x100001), FAKE, 4096, 4096, 4, 128, FAKE, None, 0, None, None) == 2
+    assert lib.qgemm(ctypes.c_void_p(0x100004), 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, 0, None, None) == 2
+    # an empty problem enqueues nothing and needs no pointers
+    assert lib.qgemm(None, 0, 0, None, None, 4096, 4096, 4, 128, None, None, 0, None, None) == 0
+    assert lib.qgemm(None, 0, 8, None, None, 0, 4096, 4, 128, None, None, 0, None, None) == 0
+
+
+def test_workspace_is_a_pure_function_of_the_problem(q4):
+    for M in (1, 4, 8, 16, 40, 300, 2048):
+        a = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)
+        b = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)
+        assert a == b and a % 256 == 0

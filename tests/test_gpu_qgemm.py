@@ -1,0 +1,186 @@
+"""qgemm on the GPU vs the oracle's fp64 matmul with the dequantized weights (the
+QuantizedMatmul of "Huit bits, puis quatre": same numbers up to summation order).
+
+Tolerance, per output element: |y_gpu - y_oracle| <= 1e-5 * sum_k |w'[n,k] x[m,k]| + 1e-6.
+The packed weights fed to the GPU come from the oracle, so this isolates the matmul.
+Full-size problems are checked on sampled output channels, computed one by one by the
+oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 1e-5, 1e-6
+
+
+@pytest.fixture(scope="module")
+def q4():
+    import int4_quantized_b200 as m
+
+    m.lib()
+    return m
+
+
+def run_gpu(q4, x, payload, scales, N, K, bits, group, bf16=False):
+    import torch
+
+    xt = torch.from_numpy(x).cuda()
+    if bf16:
+        xt = xt.to(torch.bfloat16)
+    y = q4.qgemm(xt, torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda(), N, K, bits, group)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def check(y, yref, bound, what):
+    err = np.abs(y.astype(np.float64) - yref)
+    lim = RTOL * bound + ATOL
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, f"{what}: {len(bad)} outside tolerance, worst ratio {float((err / lim).max()):.3g} at {bad[:3].tolist()}"
+    return float((err / lim).max())
+
+
+def sample_rows(N, k, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(16, N))) | set(range(max(0, N - 16), N))
+    rows |= set(rng.choice(N, min(k, N), replace=False).tolist())
+    return sorted(rows)
+
+
+def case(q4, w, x, bits, group, rows=None, bf16=False, what=""):
+    N, K = w.shape
+    payload, scales, _ = oracle.pack(w, bits, group)
+    xin = x
+    if bf16:
+        import torch
+
+        xin = torch.from_numpy(x).to(torch.bfloat16).float().numpy()  # the values the GPU sees
+    y = run_gpu(q4, x, payload, scales, N, K, bits, group, bf16=bf16)
+    assert y.shape == (x.shape[0], N)
+    yref, bound = oracle.qgemm(xin, payload, scales, N, K, bits, group, rows=rows)
+    ysel = y if rows is None else y[:, rows]
+    assert np.all(np.isfinite(y))
+    return check(ysel, yref, bound, what)
+
+
+def test_small_config_full(q4):
+    wl = workloads.WORKLOADS["small"]
+    w = workloads.weight(wl.matrices[0])
+    x = workloads.activations(1, 1024, wl.x_seed(1024))
+    for bits, g in wl.formats:
+        case(q4, w, x, bits, g, what=f"small int{bits} g{g}")
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_mid_config_full(q4, M):
+    wl = workloads.WORKLOADS["mid"]
+    w = workloads.weight(wl.matrices[0])
+    x = workloads.activations(M, 4096, wl.x_seed(4096))
+    for bits, g in wl.formats:
+        case(q4, w, x, bits, g, what=f"mid int{bits} g{g} M{M}")
+
+
+@pytest.mark.parametrize("idx", [0, 4, 6])   # q (4096x4096), gate (11008x4096), down (4096x11008)
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_llama7b_sampled(q4, idx, M):
+    wl = workloads.WORKLOADS["llama7b"]
+    m = wl.matrices[idx]
+    w = workloads.weight(m)
+    x = workloads.activations(M, m.K, wl.x_seed(m.K))
+    rows = sample_rows(m.N, 200, idx)
+    for bits, g in wl.formats:
+        case(q4, w, x, bits, m.K if g is None else g, rows=rows, what=f"{m.name} int{bits} M{M}")
+
+
+@pytest.mark.parametrize("which", [0, 2])
+def test_mlp70b_sampled(q4, which):
+    wl = workloads.WORKLOADS["mlp70b"]
+    m = wl.matrices[which]
+    w = workloads.weight(m)
+    x = workloads.activations(1, m.K, wl.x_seed(m.K))
+    case(q4, w, x, 4, 64, rows=sample_rows(m.N, 300, which), what=m.name)
+
+
+@pytest.mark.parametrize("M", [1, 9, 40, 300])
+def test_row_counts(q4, M):
+    # the codes path is checked for 1, 9, 40 and 300 activation rows ("Huit bits, puis
+    # quatre", section "Ranger des entiers dans des f32")
+    rng = np.random.default_rng(M)
+    w = rng.normal(0, 0.02, (512, 1024)).astype(np.float32)
+    x = rng.normal(0, 1, (M, 1024)).astype(np.float32)
+    for bits, g in ((4, 128), (8, 1024), (4, 32), (8, 64)):
+        case(q4, w, x, bits, g, what=f"M{M} int{bits} g{g}")
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (4, 128), (4, 256), (4, 4096),
+                                        (8, 16), (8, 32), (8, 64), (8, 128), (8, 4096)])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 13, 16])
+def test_group_variants(q4, bits, group, M):
+    rng = np.random.default_rng(bits * 1000 + group + M)
+    N, K = 200, 4096  # ragged N: not a multiple of 16
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    w.reshape(-1)[rng.choice(N * K, 50, replace=False)] *= 20  # outliers
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    case(q4, w, x, bits, group, what=f"int{bits} g{group} M{M}")
+
+
+@pytest.mark.parametrize("M", [1, 16, 40, 64, 128])
+def test_bf16_activations(q4, M):
+    rng = np.random.default_rng(77 + M)
+    w = rng.normal(0, 0.02, (384, 2048)).astype(np.float32)
+    x = rng.normal(0, 1, (M, 2048)).astype(np.float32)
+    for bits, g in ((4, 128), (8, 2048)):
+        case(q4, w, x, bits, g, bf16=True, what=f"bf16 M{M} int{bits}")
+
+
+def test_activation_range_extremes(q4):
+    # tiny, huge and mixed-magnitude activations: the exact fp16 split rescales by 2^-e
+    rng = np.random.default_rng(5)
+    w = rng.normal(0, 0.02, (64, 512)).astype(np.float32)
+    for scale in (1e-30, 1e-8, 1e-3, 1e4, 1e30):
+        x = (rng.normal(0, 1, (3, 512)) * scale).astype(np.float32)
+        case(q4, w, x, 4, 128, what=f"x scale {scale}")
+    x = rng.normal(0, 1, (2, 512)).astype(np.float32)
+    x[0, :256] *= 1e-12
+    x[1, 7] = 6.0e4
+    case(q4, w, x, 8, 64, what="mixed magnitudes")
+    x = np.zeros((2, 512), np.float32)
+    case(q4, w, x, 4, 128, what="zeros")
+
+
+def test_one_hot_selects_dequantized_weight_exactly(q4):
+    # with x = e_k the only product is code * 1, scaled once by the fp32 scale:
+    # y[:, n] equals w'[n, k] bit for bit
+    wl = workloads.WORKLOADS["mid"]
+    w = workloads.weight(wl.matrices[0])
+    for bits, g in wl.formats:
+        payload, scales, _ = oracle.pack(w, bits, g)
+        for k in (0, 1, 127, 4095):
+            x = np.zeros((1, 4096), np.float32)
+            x[0, k] = 1.0
+            y = run_gpu(q4, x, payload, scales, 4096, 4096, bits, g)
+            col = oracle.dequant_rows(payload, scales, 4096, 4096, bits, g)[:, k]
+            assert np.array_equal(y[0].view(np.uint32), col.view(np.uint32)), (bits, k)
+
+
+def test_empty_shapes(q4):
+    import torch
+
+    p = torch.zeros(64 * 64, dtype=torch.uint8, device="cuda")
+    s = torch.ones(64 * 64 // 32, dtype=torch.float32, device="cuda")
+    y = q4.qgemm(torch.zeros((0, 128), device="cuda"), p, s, 64, 128, 4, 32)
+    assert y.shape == (0, 64)
+
+
+def test_deterministic(q4):
+    rng = np.random.default_rng(9)
+    w = rng.normal(0, 0.02, (4096, 4096)).astype(np.float32)
+    x = rng.normal(0, 1, (8, 4096)).astype(np.float32)
+    payload, scales, _ = oracle.pack(w, 4, 128)
+    a = run_gpu(q4, x, payload, scales, 4096, 4096, 4, 128)
+    b = run_gpu(q4, x, payload, scales, 4096, 4096, 4, 128)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
