@@ -111,10 +111,11 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
                    int bits, int64_t group, float *w_out, void *stream);
 
 /*
- * Workspace bytes that qgemm needs for this problem (0 when it needs none, which
- * is the case for every shape the decode GEMV takes). Same arguments as qgemm.
- * Returns 0 also for arguments qgemm rejects. Depends only on the arguments, not
- * on the device.
+ * Workspace bytes that qgemm needs for this problem: the activations converted
+ * once into tensor-core fragment order (about 16 bytes per element of x for up
+ * to 4 rows of x, 64 per row beyond) plus one exponent per row of x and block of
+ * 2048 k. Same arguments as qgemm. Returns 0 for arguments qgemm rejects.
+ * Depends only on the arguments, not on the device.
  */
 Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt);
@@ -130,10 +131,9 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  *   scales   [N*K/group] floats from the same qpack
  *   y        out, [M][N] fp32
  *   workspace  device scratch of at least q4_qgemm_workspace_bytes(...)
- *            bytes, 256-byte aligned, owned by the caller; may be NULL when
- *            that size is 0. Its contents need no initialisation and are
- *            meaningless after the call. Two calls that may run at the same
- *            time must not share a workspace.
+ *            bytes, 256-byte aligned, owned by the caller. Its contents need
+ *            no initialisation and are meaningless after the call. Two calls
+ *            that may run at the same time must not share a workspace.
  *   status_word  optional (may be NULL) device uint32. Every wait inside the
  *            kernels is bounded; if one ever gives up, Q4_STATUS_TIMEOUT is
  *            OR-ed into this word and y must be treated as invalid. The

@@ -123,7 +123,7 @@ q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
     if ((uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return Q4_ERR_WORKSPACE;
     cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,
-                                    status_word, as_stream(stream));
+                                    workspace, status_word, as_stream(stream));
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 

@@ -109,25 +109,34 @@ Q4_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps in
+// hardware (up to ~1 ms per call) and wakes when the phase completes, instead of
+// spinning and stealing issue slots from the warps that do the math.
 Q4_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after ~2^22 polls with back-off (well over a second), so a
-// lost arrival can never hang the GPU. Returns false on timeout.
+Q4_DEVINL uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait: retries the suspending try_wait; the global timer bounds the whole wait
+// at about one second, so a lost arrival can never hang the GPU. Returns false on timeout.
 Q4_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < (1u << 22); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (i > 64) __nanosleep(256);
+        if (global_ns() - t0 > 1000000000ull) return false;
     }
-    return false;
 }
 // 2D tiled TMA load global -> shared, completion counted in bytes on `bar`.
 Q4_DEVINL void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int c0, int c1) {
@@ -136,8 +145,25 @@ Q4_DEVINL void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int c0, i
         ::"r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
+// 4-byte asynchronous copy global -> shared (no register staging, no load-use stall).
+Q4_DEVINL void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (counts as one
+// of the barrier's expected arrivals).
+Q4_DEVINL void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 Q4_DEVINL void named_barrier_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// D = A * B with a zero accumulator (starts a new sum without zeroing registers).
+Q4_DEVINL void mma_f16_16816_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
 }  // namespace q4

@@ -18,23 +18,23 @@ cudaError_t launch_qdequant(const uint8_t *payload, const float *scales, int64_t
 // Plan of one GEMV call: how K is cut into segments (one 128/64/32-bit load per lane per
 // weight row), how a thread-block cluster splits K, and how much x is staged at a time.
 struct GemvPlan {
-    int bits, L;       // L = bytes each lane loads per weight row per segment (16, 8 or 4)
-    int segk;          // k per segment = 32 * L / bits
-    int segs;          // segments per row = K / segk
-    int spg;           // segments per scale group = group / segk
-    int NB;            // n8 blocks of activation columns per 16-row chunk of x (1, 2 or 4)
-    int D;             // unused (0)
-    int T;             // 16-row tiles of W = ceil(N / 16)
-    int clusters;      // CTAs along N = ceil(N / 128)
-    int CS;            // CTAs per cluster = splits of K (1, 2, 4 or 8)
-    int stages_total;  // 128-byte tiles per weight row
-    int stages_per_cta;// tiles per CTA's K range
-    int phase_stages;  // tiles of x staged in shared memory at a time
-    int seg_per_cta;   // segments per CTA's K range
-    int phase_segs;    // segments of x staged at a time
-    int nmc;           // 16-row chunks of x = ceil(M / 16)
-    size_t smem_bytes; // dynamic shared memory per CTA
-    size_t bytes;      // global workspace bytes (0: the GEMV needs none)
+    int bits, L;        // L = bytes each lane reads per weight row per segment (16, 8 or 4)
+    int segk;           // k per segment = 32 * L / bits
+    int segs;           // segments per row = K / segk
+    int spg;            // segments per scale group = group / segk
+    int NB;             // n8 blocks of activation columns per 16-row chunk of x (1, 2 or 4)
+    int lw;             // fragment lanes stored per (k-tile, n8 block)
+    int T;              // 16-row tiles of W = ceil(N / 16)
+    int clusters;       // CTAs along N = ceil(N / 128)
+    int CS;             // CTAs per cluster = splits of K (1..8)
+    int stages_total;   // 128-byte tiles per weight row
+    int stages_per_cta; // tiles per CTA's K range
+    int ebs, n_eb;      // tiles per k-block (exponent and scale block), k-blocks per row
+    int nst_ring;       // ring depth
+    int slot_bytes;     // bytes of one ring slot
+    int nmc;            // 16-row chunks of x = ceil(M / 16)
+    size_t smem_bytes;  // dynamic shared memory per CTA
+    size_t off_frag, off_exp, bytes;  // workspace layout and size
 };
 
 // Returns false when this GEMV does not cover (bits, group, K).
@@ -42,6 +42,6 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
 
 cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t M,
                         const uint8_t *payload, const float *scales, int64_t N, int64_t K,
-                        int64_t group, float *y, uint32_t *status, cudaStream_t st);
+                        int64_t group, float *y, void *ws, uint32_t *status, cudaStream_t st);
 
 }  // namespace q4

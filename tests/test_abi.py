@@ -89,14 +89,17 @@ def test_qgemm_validation(q4, M, N, K, bits, group, xt, expect):
 
 def test_qgemm_workspace_rules(q4):
     lib = q4.lib()
-    # the decode GEMV needs no global scratch at all
-    for M in (1, 8, 16, 40):
-        assert lib.q4_qgemm_workspace_bytes(M, 4096, 4096, 4, 128, 0) == 0
-    # a workspace that is given must be 256-byte aligned
-    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ctypes.c_void_p(0x100010), 1 << 20, None, None) == 5
+    need = lib.q4_qgemm_workspace_bytes(8, 4096, 4096, 4, 128, 0)
+    assert need > 0 and need % 256 == 0
+    # one row of x needs less fragment space than four
+    assert lib.q4_qgemm_workspace_bytes(1, 4096, 4096, 4, 128, 0) < lib.q4_qgemm_workspace_bytes(4, 4096, 4096, 4, 128, 0)
+    ok = ctypes.c_void_p(0x100000)
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need - 1, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ctypes.c_void_p(0x100010), need, None, None) == 5
     # misaligned payload / x are reported before anything is enqueued
-    assert lib.qgemm(FAKE, 0, 8, ctypes.c_void_p(0x100001), FAKE, 4096, 4096, 4, 128, FAKE, None, 0, None, None) == 2
-    assert lib.qgemm(ctypes.c_void_p(0x100004), 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, 0, None, None) == 2
+    assert lib.qgemm(FAKE, 0, 8, ctypes.c_void_p(0x100001), FAKE, 4096, 4096, 4, 128, FAKE, ok, need, None, None) == 2
+    assert lib.qgemm(ctypes.c_void_p(0x100004), 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need, None, None) == 2
     # an empty problem enqueues nothing and needs no pointers
     assert lib.qgemm(None, 0, 0, None, None, 4096, 4096, 4, 128, None, None, 0, None, None) == 0
     assert lib.qgemm(None, 0, 8, None, None, 0, 4096, 4, 128, None, None, 0, None, None) == 0
