@@ -51,7 +51,9 @@ typedef enum q4_status {
     Q4_ERR_UNSUPPORTED = 2, /* a valid format that this kernel does not cover (see each call) */
     Q4_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
     Q4_ERR_NONFINITE = 4,   /* qpack saw Inf or NaN (reported through its status word) */
-    Q4_ERR_WORKSPACE = 5    /* qgemm workspace null, too small or not 256-byte aligned */
+    Q4_ERR_WORKSPACE = 5,   /* qgemm workspace null, too small or not 256-byte aligned */
+    Q4_ERR_SCRATCH_LIMIT = 6 /* qgemm_noalloc: the problem needs more than
+                               Q4_NOALLOC_SCRATCH_BYTES of scratch */
 } q4_status;
 
 typedef enum q4_xdtype {
@@ -151,6 +153,35 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
 Q4_API q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
                 const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
                 void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream);
+
+/* Size of the one device scratch buffer that qgemm_noalloc uses (4 MiB). */
+#define Q4_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * qgemm_noalloc -- qgemm without a caller workspace and without any device
+ * allocation in the call. The pages have no counterpart: this is an interface
+ * convenience for callers that must not allocate (e.g. code running under a
+ * memory budget fixed up front). The result is the same as qgemm's.
+ *   Arguments as qgemm, minus workspace and workspace_bytes.
+ *   Scratch: a file-scope device array of Q4_NOALLOC_SCRATCH_BYTES inside
+ *            libq4, one per device, created by the CUDA runtime with the
+ *            library's module. The first call on each device (with that device
+ *            current) looks up its address once and caches it; make that first
+ *            call before any stream capture on the device. Nothing in the
+ *            scratch has to start at zero: each call writes every byte it reads.
+ *   Limit:   problems with q4_qgemm_workspace_bytes(...) greater than
+ *            Q4_NOALLOC_SCRATCH_BYTES are rejected with Q4_ERR_SCRATCH_LIMIT
+ *            before anything is enqueued (M <= 16 fits for K up to about 60000).
+ *   Concurrency: every call on a device shares the one scratch, so two calls
+ *            that may overlap on the GPU (different streams with no ordering
+ *            between them) race and give wrong results. Calls on one stream,
+ *            or otherwise ordered, are safe.
+ * Errors: those of qgemm except Q4_ERR_WORKSPACE, plus Q4_ERR_SCRATCH_LIMIT;
+ * Q4_ERR_CUDA also when the scratch address cannot be obtained.
+ */
+Q4_API q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                uint32_t *status_word, void *stream);
 
 #ifdef __cplusplus
 }

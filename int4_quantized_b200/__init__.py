@@ -24,11 +24,13 @@ import torch
 
 __all__ = [
     "Q4Error", "lib", "lib_path", "payload_bytes", "num_scales", "qgemm_workspace_bytes",
-    "qpack", "qdequant", "qgemm", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
-    "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_X_F32", "Q4_X_BF16", "STATUS_NONFINITE", "STATUS_TIMEOUT",
+    "qpack", "qdequant", "qgemm", "qgemm_noalloc", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
+    "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_ERR_SCRATCH_LIMIT", "Q4_X_F32", "Q4_X_BF16", "STATUS_NONFINITE", "STATUS_TIMEOUT",
 ]
 
-Q4_OK, Q4_ERR_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_CUDA, Q4_ERR_NONFINITE, Q4_ERR_WORKSPACE = range(6)
+Q4_OK, Q4_ERR_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_CUDA, Q4_ERR_NONFINITE, Q4_ERR_WORKSPACE, \
+    Q4_ERR_SCRATCH_LIMIT = range(7)
+NOALLOC_SCRATCH_BYTES = 4 << 20  # Q4_NOALLOC_SCRATCH_BYTES
 Q4_X_F32, Q4_X_BF16 = 0, 1
 STATUS_NONFINITE = 1
 STATUS_TIMEOUT = 2
@@ -71,6 +73,8 @@ def lib() -> ctypes.CDLL:
                 L.q4_qgemm_workspace_bytes.restype = sz
                 L.qgemm.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, sz, vp, vp]
                 L.qgemm.restype = i32
+                L.qgemm_noalloc.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, vp]
+                L.qgemm_noalloc.restype = i32
                 _lib = L
     return _lib
 
@@ -187,4 +191,28 @@ def qgemm(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, N: int, 
     with torch.cuda.device(x.device):
         _check(lib().qgemm(_ptr(x2), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group, _ptr(out),
                            _ptr(workspace), ws_bytes, _ptr(status), _stream(x.device)), "qgemm")
+    return out
+
+
+def qgemm_noalloc(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, N: int, K: int,
+                  bits: int, group: int, out: torch.Tensor, status: Optional[torch.Tensor] = None
+                  ) -> torch.Tensor:
+    """qgemm into a caller-given `out` using the library's built-in device scratch.
+
+    Allocates nothing. All calls on one device share that scratch, so calls that may
+    overlap on the GPU race; calls on one stream are safe.
+    """
+    _cuda(x, "x")
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _cuda(payload, "payload", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    _cuda(out, "out", torch.float32)
+    M = x.numel() // K if K else 0
+    xt = Q4_X_BF16 if x.dtype == torch.bfloat16 else Q4_X_F32
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    with torch.cuda.device(x.device):
+        _check(lib().qgemm_noalloc(_ptr(x), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group,
+                                   _ptr(out), _ptr(status), _stream(x.device)), "qgemm_noalloc")
     return out

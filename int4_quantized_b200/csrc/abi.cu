@@ -1,9 +1,11 @@
 // abi.cu -- the extern "C" entry points declared in include/q4.h.
 //
 // Every call validates its arguments on the host before enqueuing anything, then
-// launches the kernels on the caller's stream. Nothing is allocated here and no state
-// survives a call.
+// launches the kernels on the caller's stream. Nothing is allocated here; the only state
+// that survives a call is qgemm_noalloc's cached scratch address per device.
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "kernels.h"
 
@@ -49,6 +51,28 @@ q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q
     return Q4_OK;
 }
 
+// Scratch of qgemm_noalloc: one file-scope device array per device, created with the
+// module; its address is looked up once per device and cached.
+constexpr size_t kNoAllocBytes = Q4_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+q4_status noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return Q4_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return Q4_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return Q4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -63,6 +87,7 @@ const char *q4_status_str(q4_status s) {
         case Q4_ERR_CUDA: return "CUDA error";
         case Q4_ERR_NONFINITE: return "non-finite weight in a group";
         case Q4_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case Q4_ERR_SCRATCH_LIMIT: return "problem needs more scratch than qgemm_noalloc's built-in buffer";
     }
     return "unknown status";
 }
@@ -125,6 +150,21 @@ q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
     cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,
                                     workspace, status_word, as_stream(stream));
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                        const float *scales, int64_t N, int64_t K, int bits, int64_t group,
+                        float *y, uint32_t *status_word, void *stream) {
+    q4::GemvPlan pl;
+    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &pl);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (pl.bytes > kNoAllocBytes) return Q4_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != Q4_OK) return st;
+    return qgemm(x, xt, M, payload, scales, N, K, bits, group, y, scratch, kNoAllocBytes,
+                 status_word, stream);
 }
 
 }  // extern "C"
