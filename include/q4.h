@@ -113,11 +113,13 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
                    int bits, int64_t group, float *w_out, void *stream);
 
 /*
- * Workspace bytes that qgemm needs for this problem: the activations converted
- * once into tensor-core fragment order (about 16 bytes per element of x for up
- * to 4 rows of x, 64 per row beyond) plus one exponent per row of x and block of
- * 2048 k. Same arguments as qgemm. Returns 0 for arguments qgemm rejects.
- * Depends only on the arguments, not on the device.
+ * Workspace bytes that qgemm needs for this problem: with two or more rows of
+ * x, the activations converted once into fixed-point digits in tensor-core
+ * fragment order (4 bytes per element of x, rows padded to pairs and 16-row
+ * chunks) plus one exponent per row of x and block of up to 1024 k. One row
+ * of x needs none (0) when each CTA's share of K fits on chip, which holds up
+ * to K = 8192 per CTA. Same arguments as qgemm. Returns 0 for arguments qgemm
+ * rejects. Depends only on the arguments, not on the device.
  */
 Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt);
@@ -145,8 +147,8 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
  * finite inputs (y_exact = the fp64 sum).
  * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0, group divides K and
- * group % 32 == 0 (per-channel scales are group = K); for int8 group % 16
- * == 0 suffices. M, N >= 0; M == 0 or N == 0 enqueues nothing.
+ * group % 32 == 0 (per-channel scales are group = K). M, N >= 0; M == 0 or
+ * N == 0 enqueues nothing.
  * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
  * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
  */

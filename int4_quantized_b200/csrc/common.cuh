@@ -149,6 +149,10 @@ Q4_DEVINL void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int c0, i
 Q4_DEVINL void cp_async4(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+// 16-byte asynchronous copy global -> shared (both addresses 16-byte aligned), L2 only.
+Q4_DEVINL void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 // Arrive on `bar` once this thread's earlier cp.async copies have landed (counts as one
 // of the barrier's expected arrivals).
 Q4_DEVINL void cp_async_arrive(uint64_t *bar) {
@@ -164,6 +168,27 @@ Q4_DEVINL void mma_f16_16816_z(float (&c)[4], const uint32_t (&a)[4], uint32_t b
         "{%10,%10,%10,%10};"
         : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// ---- tensor cores (warp-level MMA, A/B int8, exact int32 accumulate) -----------------
+// D[16x8] (+)= A[16x32] * B[32x8], lane = 4*g + t:
+//   a0: (row g,   k 4t..4t+3)     a1: (row g+8, k 4t..4t+3)
+//   a2: (row g,   k 4t+16..4t+19) a3: (row g+8, k 4t+16..4t+19)
+//   b0: (k 4t..4t+3, col g)       b1: (k 4t+16..4t+19, col g)
+//   c0c1: (row g, col 2t..2t+1)   c2c3: (row g+8, col 2t..2t+1)
+Q4_DEVINL void mma_s8_16832(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A * B with a zero accumulator (starts a new exact sum without clearing registers).
+Q4_DEVINL void mma_s8_16832_z(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
 }
 
 }  // namespace q4

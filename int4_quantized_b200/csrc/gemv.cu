@@ -3,38 +3,43 @@
 // y[m][n] = sum_k x[m][k] * w'[n][k], w' = code * scale (pack()/unpack() of the
 // "量化推理" page; the QuantizedMatmul of "Huit bits, puis quatre", which reads the
 // codes in generation products, where one waits on memory). The packed weights are the
-// whole cost, so the kernel is built around streaming them:
+// whole cost, so the kernel is built around streaming them with as few instructions per
+// byte as possible.
 //
-//   gemv_prep   (tiny grid) turns x into tensor-core B fragments once per call: every
-//               activation row m is split exactly into x' = hi + lo (two fp16 values,
-//               22 significant bits) after a power-of-two rescale x' = x * 2^-e whose e is
-//               chosen per (m, block of k) so that the block maximum lands in
-//               [2^14, 2^15); the fragments go to a global workspace in the exact order
-//               the MMA wants them, the exponents next to them.
-//   gemv_stream (one wave: up to two CTAs per SM) streams the codes. A producer warp
-//               issues, per stage, one 2D TMA load of a 128-row x 128-byte tile of the
-//               payload (128-byte swizzle) plus one bulk copy of the matching fragment
-//               tile into a 4-deep shared-memory ring guarded by full/empty mbarriers,
-//               and loads each k-block's scales into double-buffered shared memory one
-//               block ahead. Eight consumer warps decode and multiply; they do no
-//               staging work of their own. It is launched as a programmatic dependent
-//               of gemv_prep: the payload loads start before the fragments exist, and
-//               only the fragment copies wait (griddepcontrol.wait).
+// Arithmetic: exact integer dot products on the tensor cores (warp-level mma.sync
+// m16n8k32, s8 x s8 -> s32).
+//   A = 16 weight rows x 32 k of codes as int8: int8 codes as they are stored; int4
+//       nibbles u = code + 8 become the byte 16 * code with one mask-and-xor (high
+//       nibble) or shift-mask-xor (low nibble), so a 32-bit word of 8 codes costs three
+//       logic instructions. The factor 16 is an exact power of two folded in at the end.
+//   B = 32 k x 8 columns of activation digits: each activation row m is written, per
+//       block of k, as the 32-bit fixed-point value X = rint(x * 2^(30-E)) (E chosen so
+//       that max|x| over the block is below 2^E) and X is split into four balanced
+//       base-256 digits in [-128, 127]; one B column per digit.
+//   C = int32, exact: the products and their sums within a scale group are integers.
+// When a scale group ends (or a 128-byte stage ends) each lane combines its two digit
+// columns 256*c0 + c1 (still exact), converts once to fp32, multiplies by the group's
+// fp32 scale and accumulates in fp32; the block's 2^(E-30) (and 2^16 for the high digit
+// pair) is applied exactly when the k-block ends. The only roundings are the fixed-point
+// activation (2^-31 of the block maximum) and the fp32 sums of the group results.
 //
-// Tensor cores (warp-level mma.sync m16n8k16, fp16 operands, fp32 accumulation):
-//   A = 16 weight rows x 16 k of CODES, exact in fp16 (|code| <= 127).
-//   B = 16 k x 8 columns: columns 2c and 2c+1 hold hi and lo of one activation row,
-//       so one lane owns both partial sums of the same (weight row, m) in c0/c1.
-//   When a scale group ends, the lane multiplies the partial sum by the group's fp32
-//   scale and adds it to an fp32 accumulator; no arithmetic on w' is done in fp16. At
-//   the end of each k-block the block's 2^e is applied exactly.
-// Inside a group the order of k is permuted so that a lane builds its A fragment from
-// one shared-memory read; the fragments use the same permutation. Rows are permuted
-// inside each 16-row tile so those reads are free of bank conflicts.
-//
-// A thread-block cluster of CS CTAs splits K; the CS partial sums meet in distributed
-// shared memory (fixed rank order), so results do not depend on timing. Every wait is
-// bounded; one that gives up sets Q4_STATUS_TIMEOUT in the optional status word.
+// Structure (one wave: up to two CTAs per SM, a thread-block cluster of CS CTAs splits K):
+//   a producer warp issues, per stage, one 2D TMA load of a 128-row x 128-byte tile of
+//   the payload (128-byte swizzle) into a shared-memory ring guarded by full/empty
+//   mbarriers, and loads each k-block's scales into double-buffered shared memory with
+//   asynchronous copies (16 bytes wide when the rows of scales allow) one block ahead;
+//   eight consumer warps decode and multiply.
+//   One activation row (the decode case): the consumers build the digits of their CTA's
+//   K range into shared memory while the first payload tiles are in flight; there is no
+//   second kernel and no workspace.
+//   Several rows: gemv_prep writes the digits once into the caller's workspace, in MMA
+//   order, and the stream kernel (its programmatic dependent) copies each stage's tile
+//   with a bulk copy into a second ring; the payload loads start before gemv_prep ends.
+// Inside a group the order of k is permuted so that a lane builds its A fragment from its
+// own shared-memory words; the digits use the same permutation. Rows are permuted inside
+// each 16-row tile so those reads are free of bank conflicts. The CS partial sums of a
+// cluster meet in distributed shared memory in fixed rank order, so results do not depend
+// on timing. Every wait is bounded; one that gives up sets Q4_STATUS_TIMEOUT.
 #include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched at run time)
 
 #include "common.cuh"
@@ -51,25 +56,36 @@ constexpr int kRowsPerCta = 16 * kConsumers;       // 128
 constexpr int kTileBytes = 128;                    // bytes of a weight row per stage
 constexpr int kPayloadBytes = kTileBytes * kRowsPerCta;  // 16 KB of codes per stage
 constexpr int kMaxStages = 6;
-constexpr int kSG = 17;                            // scale slots per row per k-block (odd)
+constexpr int kGroupsPerBlock = 8;                 // scale groups per k-block (target)
+constexpr int kBlockK = 1024;                      // at most k per k-block
+constexpr int kSG = 12;                            // scale slots per row per k-block (<= 9 used,
+                                                   // + up to 3 to keep 16-byte copies aligned)
+constexpr int kMaxLocalBlocks = 40;                // k-blocks one CTA may touch (in-kernel digits)
+constexpr int kFragCap = 32768;                    // in-kernel digit bytes (4 per k)
+constexpr int kSmemBudget = 115200;                // two CTAs per SM
+constexpr int kRedBytes = kRowsPerCta * 16 * 4;    // cluster partial sums, aliased on the ring
 
 struct GemvArgs {
     const float *scales;
     const void *x;
     float *y;
     uint32_t *status;
-    const uint8_t *frag;  // global fragments: [mc][k-tile][nb][LW lanes] x uint2
-    int *ebexp;           // exponents: [mc*16 + m][n_eb]
+    uint8_t *frag;        // workspace digits: [mc][stage][fslot_bytes] (several rows of x)
+    int *ebexp;           // workspace exponents: [mc*16 + m][n_eb]
     int M, N, K;
-    int segs, spg, scales_per_row;
+    int segs;             // segments per weight row
+    int spg;              // segments per scale group
+    int scales_per_row;   // K / group
     int CS;               // CTAs per cluster = K splits
     int stages_total;     // 128-byte tiles per weight row (last may be partial)
     int stages_per_cta;
-    int ebs;              // stages per k-block (exponent + scale block)
+    int ebs;              // stages per k-block (exponent and scale block)
     int n_eb;
-    int lw;               // fragment lanes stored per (k-tile, nb): 8*M for one block of <= 4 rows, else 32
-    int nst_ring;         // stages in the ring (<= kMaxStages)
-    int slot_bytes;       // payload + fragment bytes of one ring slot (1024-aligned)
+    int lw;               // digit lanes per (MMA, n8 block): 16 for one row of x, else 32
+    int NB;               // n8 blocks per 16-row chunk of x (2 rows of x per block)
+    int paired;           // digits of two consecutive MMAs interleaved (16-byte reads)
+    int nst_ring;         // ring depth
+    int fslot_bytes;      // digit bytes of one stage
 };
 
 // ---- small PTX helpers for clusters --------------------------------------------------
@@ -83,174 +99,186 @@ Q4_DEVINL float ld_dsmem_f32(const float *local_smem_ptr, uint32_t rank) {
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r));
     return v;
 }
+Q4_DEVINL void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 
-template <bool XBF16>
-Q4_DEVINL void load_x4(const void *x, int64_t idx, float (&v)[4]) {
-    if constexpr (XBF16) {
-        const uint2 b = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(x) + idx);
-        v[0] = __uint_as_float(b.x << 16);
-        v[1] = __uint_as_float(b.x & 0xffff0000u);
-        v[2] = __uint_as_float(b.y << 16);
-        v[3] = __uint_as_float(b.y & 0xffff0000u);
+// ---- activation digits --------------------------------------------------------------
+Q4_DEVINL float pow2(int e) { return __int_as_float((e + 127) << 23); }  // 2^e, e in [-126, 127]
+
+// v * 2^e in two exact power-of-two steps (e may leave [-126, 127]); one rounding at most,
+// and only when the result is subnormal.
+Q4_DEVINL float scale2(float v, int e) {
+    const int e1 = min(max(e, -126), 127);
+    const int e2 = min(max(e - e1, -126), 127);
+    return (v * pow2(e1)) * pow2(e2);
+}
+
+// E such that every |x| of a block is below 2^E, from the bits of the block's max |x|;
+// 0 for an all-zero (or non-finite) block.
+Q4_DEVINL int block_exp(uint32_t mx) {
+    if (mx == 0 || mx >= 0x7f800000u) return 0;
+    const int be = (int)(mx >> 23);
+    if (be > 0) return be - 126;
+    return (32 - __clz((int)mx)) - 149;  // subnormal: mx * 2^-149 with mx < 2^23
+}
+
+// Balanced base-256 digits of X = rint(v * 2^(30-E)) (|X| < 2^30), packed with the least
+// significant digit in byte 0: X = sum_p digit_p * 256^p, every digit in [-128, 127].
+// (X + 0x808080) has unsigned low bytes b_p; digit_p = b_p - 128, i.e. b_p ^ 0x80.
+Q4_DEVINL uint32_t digits4(float v, float f1, float f2) {
+    const int X = __float2int_rn((v * f1) * f2);
+    return (uint32_t)(X + 0x00808080) ^ 0x00808080u;
+}
+
+// out[p] = byte p of (a, b, c, d), in that order.
+Q4_DEVINL void transpose4(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t (&out)[4]) {
+    const uint32_t t0 = prmt(a, b, 0x5140u), t1 = prmt(a, b, 0x7362u);
+    const uint32_t t2 = prmt(c, d, 0x5140u), t3 = prmt(c, d, 0x7362u);
+    out[0] = prmt(t0, t2, 0x5410u);
+    out[1] = prmt(t0, t2, 0x7632u);
+    out[2] = prmt(t1, t3, 0x5410u);
+    out[3] = prmt(t1, t3, 0x7632u);
+}
+
+// Index (uint2 units) of the B fragment of MMA i of a stage, n8 block nb, lane.
+Q4_DEVINL int frag_idx(int i, int nb, int lane, int NB, int lw, bool paired) {
+    return paired ? ((((i >> 1) * NB + nb) * lw + lane) << 1) + (i & 1) : (i * NB + nb) * lw + lane;
+}
+
+// The B fragments of 8 consecutive k (offset kk inside the stage, a multiple of 8) of
+// activation row m of a 16-row chunk. Column 4h + (3 - p) of n8 block m/2 (h = m % 2)
+// holds digit p, so a lane's accumulator pair (c0, c1) is (digit 3, digit 2) for t even
+// and (digit 1, digit 0) for t odd: 256 * c0 + c1 is the high / low half of the sum.
+// k-slots of the MMA (PTX m16n8k32 layout) map onto memory k as the lane's A words do:
+// int4: b0 = the even k of the word, b1 = the odd k; int8: b0 = k 0..3, b1 = k 4..7.
+template <int BITS, int L>
+Q4_DEVINL void frag_unit(uint2 *stage, int kk, int m, const float (&v)[8], float f1, float f2, int NB,
+                         int lw, bool paired) {
+    constexpr int KTI = BITS == 4 ? L / 4 : L / 8;  // MMAs per segment
+    const int byte = BITS == 4 ? (kk >> 1) : kk;
+    const int sl = byte / (4 * L), t = (byte % (4 * L)) / L;
+    const int j = (byte % L) / (BITS == 4 ? 4 : 8);
+    const int i = sl * KTI + j;
+    uint32_t D[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) D[q] = digits4(v[q], f1, f2);
+    uint32_t T0[4], T1[4];
+    if constexpr (BITS == 4) {
+        transpose4(D[0], D[2], D[4], D[6], T0);
+        transpose4(D[1], D[3], D[5], D[7], T1);
     } else {
-        const float4 f = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + idx);
-        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        transpose4(D[0], D[1], D[2], D[3], T0);
+        transpose4(D[4], D[5], D[6], D[7], T1);
+    }
+    const int nb = m >> 1, h = m & 1;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int lane = 16 * h + 4 * (3 - p) + t;
+        stage[frag_idx(i, nb, lane, NB, lw, paired)] = make_uint2(T0[p], T1[p]);
     }
 }
 
-// Exact split of a pair of rescaled activations into fp16 (hi, lo) pairs.
-Q4_DEVINL void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
-    const __half2 h = __floats2half2_rn(a, b);
-    const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);  // a - hf.x is exact (Sterbenz)
-    hi = *reinterpret_cast<const uint32_t *>(&h);
-    lo = *reinterpret_cast<const uint32_t *>(&l);
+template <bool XBF16>
+Q4_DEVINL void load_x8(const void *x, int64_t idx, float (&v)[8]) {
+    if constexpr (XBF16) {
+        const uint4 b = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(x) + idx);
+        const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v[2 * q] = __uint_as_float(w[q] << 16);
+            v[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + idx);
+        const float4 b = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + idx + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
 }
-Q4_DEVINL uint32_t pack_lo_halves(uint32_t p, uint32_t q) { return prmt(p, q, 0x5410u); }  // (p.x, q.x)
-Q4_DEVINL uint32_t pack_hi_halves(uint32_t p, uint32_t q) { return prmt(p, q, 0x7632u); }  // (p.y, q.y)
-Q4_DEVINL float pow2(int e) { return __int_as_float((e + 127) << 23); }  // 2^e, e in [-126, 127]
 
-// One CTA per (k-block eb, 16-row chunk mc of x): exponent per activation row, then the
-// B fragments of the block in MMA order. It lets the dependent stream kernel start at once.
-template <int BITS, int L, int NB, bool XBF16>
+Q4_DEVINL uint32_t absmax8(const float (&v)[8]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m = max(m, __float_as_uint(v[q]) & 0x7fffffffu);
+    return m;
+}
+
+// One CTA per (k-block eb, 16-row chunk mc of x): the block exponent of every activation
+// row, then the digits of the block in MMA order (several rows of x).
+template <int BITS, int L, bool XBF16>
 __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
     grid_dep_launch();
-    constexpr int SEGK = 32 * L / BITS;
-    constexpr int KT = SEGK / 16;
     constexpr int STAGEK = kTileBytes * 8 / BITS;
-    constexpr int BLK = BITS == 4 ? 8 : 4;  // k per work item
-    __shared__ uint32_t mx_sh[16];
     __shared__ int e_sh[16];
     const int eb = blockIdx.x, mc = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int mcnt = min(16, a.M - mc * 16);
     const int k0 = eb * a.ebs * STAGEK;
     const int k1 = min(a.K, k0 + a.ebs * STAGEK);
-    const int nk = k1 - k0;
-    // (a) exponent per activation row
+    const int nu = (k1 - k0) / 8;  // 8-k units in the block (at most 128)
     for (int ml = warp; ml < 16; ml += 8) {
         uint32_t mx = 0;
         if (ml < mcnt) {
             const int64_t rowb = (int64_t)(mc * 16 + ml) * a.K + k0;
-            // a k-block is at most 2048 values: 16 loads per lane, all in flight at once
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int k = lane * 4 + 128 * i;
-                if (k < nk) {
-                    float v[4];
-                    load_x4<XBF16>(a.x, rowb + k, v);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) mx = max(mx, __float_as_uint(v[q]) & 0x7fffffffu);
+            for (int r = 0; r < kBlockK / 256; ++r) {
+                const int u = lane + 32 * r;
+                if (u < nu) {
+                    float v[8];
+                    load_x8<XBF16>(a.x, rowb + 8 * u, v);
+                    mx = max(mx, absmax8(v));
                 }
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mx = __reduce_max_sync(0xffffffffu, mx);
         if (lane == 0) {
-            int e = 0;
-            if (mx != 0 && mx < 0x7f800000u) {
-                int E;
-                frexpf(__uint_as_float(mx), &E);  // max|x| in [2^(E-1), 2^E)
-                e = E - 15;                        // -> max|x| * 2^-e in [2^14, 2^15)
-            }
-            e_sh[ml] = e;
-            a.ebexp[(int64_t)(mc * 16 + ml) * a.n_eb + eb] = e;
+            const int E = block_exp(mx);
+            e_sh[ml] = E;
+            a.ebexp[(int64_t)(mc * 16 + ml) * a.n_eb + eb] = E;
         }
     }
     __syncthreads();
-    // (b) fragments of absent activation rows are zero (only the 32-lane layout has any)
-    const int64_t kt0 = k0 / 16, nkt = nk / 16;
-    uint2 *frag = reinterpret_cast<uint2 *>(const_cast<uint8_t *>(a.frag)) +
-                  ((int64_t)mc * (a.K / 16) + kt0) * NB * a.lw;
-    if (a.lw == 32 && mcnt < 4 * NB) {
-        for (int64_t i = threadIdx.x; i < nkt * NB * 32; i += blockDim.x) {
-            const int ln = (int)(i & 31), nb = (int)((i >> 5) % NB);
-            if (nb * 4 + (ln >> 3) >= mcnt) frag[i] = make_uint2(0u, 0u);
-        }
-    }
-    // (c) rescale, split, scatter into fragment order
-    const int nblk = nk / BLK;
-    for (int it = threadIdx.x; it < nblk * mcnt; it += blockDim.x) {
-        const int ml = it / nblk, blk = it - ml * nblk;
-        const int e = e_sh[ml];
-        // x * 2^-e as two exact power-of-two multiplications (2^-e may leave fp32 range)
-        const int e1 = min(max(-e, -126), 127);
-        const float f1 = pow2(e1), f2 = pow2(min(max(-e - e1, -126), 127));
-        const int64_t xb = (int64_t)(mc * 16 + ml) * a.K + k0 + blk * BLK;
+    uint2 *fbase = reinterpret_cast<uint2 *>(a.frag) + (size_t)mc * a.stages_total * (a.fslot_bytes / 8);
+    for (int it = threadIdx.x; it < nu * mcnt; it += blockDim.x) {
+        const int ml = it / nu, u = it - ml * nu;
+        const int k = k0 + 8 * u;
         float v[8];
-        {
-            float t4[4];
-            load_x4<XBF16>(a.x, xb, t4);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) v[q] = (t4[q] * f1) * f2;
-            if constexpr (BLK == 8) {
-                load_x4<XBF16>(a.x, xb + 4, t4);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) v[4 + q] = (t4[q] * f1) * f2;
-            }
-        }
-        const int kl = blk * BLK;  // k offset inside the block (blocks start on segment bounds)
-        const int sl = kl / SEGK, within = kl - sl * SEGK;
-        const int nb = ml >> 2, lane_hi = 8 * (ml & 3);
-        if constexpr (BITS == 4) {
-            // the 8 values are word w of lane quad t: k-tile 2w takes k {0,4 | 1,5},
-            // k-tile 2w+1 takes k {2,6 | 3,7}
-            const int t = within / (2 * L), w = (within % (2 * L)) / 8;
-            uint32_t h01, l01, h45, l45, h23, l23, h67, l67;
-            split2(v[0], v[1], h01, l01);
-            split2(v[4], v[5], h45, l45);
-            split2(v[2], v[3], h23, l23);
-            split2(v[6], v[7], h67, l67);
-            uint2 *f0 = frag + ((int64_t)(sl * KT + 2 * w) * NB + nb) * a.lw + lane_hi + t;
-            uint2 *f1p = f0 + NB * a.lw;  // next k-tile
-            f0[0] = make_uint2(pack_lo_halves(h01, h45), pack_hi_halves(h01, h45));
-            f0[4] = make_uint2(pack_lo_halves(l01, l45), pack_hi_halves(l01, l45));
-            f1p[0] = make_uint2(pack_lo_halves(h23, h67), pack_hi_halves(h23, h67));
-            f1p[4] = make_uint2(pack_lo_halves(l23, l67), pack_hi_halves(l23, l67));
-        } else {
-            // the 4 values are word j of lane quad t, in natural order
-            const int t = within / L, j = (within % L) / 4;
-            uint32_t h01, l01, h23, l23;
-            split2(v[0], v[1], h01, l01);
-            split2(v[2], v[3], h23, l23);
-            uint2 *f0 = frag + ((int64_t)(sl * KT + j) * NB + nb) * a.lw + lane_hi + t;
-            f0[0] = make_uint2(h01, h23);
-            f0[4] = make_uint2(l01, l23);
-        }
+        load_x8<XBF16>(a.x, (int64_t)(mc * 16 + ml) * a.K + k, v);
+        const int sh = 30 - e_sh[ml];
+        const int e1 = min(max(sh, -126), 127);
+        const float f1 = pow2(e1), f2 = pow2(min(max(sh - e1, -126), 127));
+        const int s = k / STAGEK;
+        frag_unit<BITS, L>(fbase + (size_t)s * (a.fslot_bytes / 8), k - s * STAGEK, ml, v, f1, f2, a.NB, a.lw,
+                           a.paired != 0);
     }
 }
 
 // ---- decode of the packed codes ------------------------------------------------------
-// A fragment of k-tile j from one lane's words of row g (w0) and row g+8 (w1).
+// A fragment of MMA j of a segment from one lane's words of row g (w0) and row g+8 (w1).
 template <int BITS, int L>
-Q4_DEVINL void unpack_a(uint32_t (&a)[4], const uint32_t (&w0)[L / 4], const uint32_t (&w1)[L / 4],
-                        int j) {
+Q4_DEVINL void unpack_a(uint32_t (&a)[4], const uint32_t (&w0)[L / 4], const uint32_t (&w1)[L / 4], int j) {
     if constexpr (BITS == 4) {
-        // fp16 0x6400 | u = 1024 + u; (1024 + u) - 1032 = u - 8 = code (exact)
-        // fp16 0x6400 | (u << 4) = 1024 + 16u; (1024 + 16u) / 16 - 72 = code (exact)
-        const uint32_t kMagic = 0x64006400u, kSub = 0x64086408u /* 1032 */;
-        const uint32_t kInv16 = 0x2c002c00u /* 1/16 */, kNeg72 = 0xd480d480u /* -72 */;
-        uint32_t x0 = w0[j >> 1], x1 = w1[j >> 1];
-        if (j & 1) { x0 >>= 8; x1 >>= 8; }
-        a[0] = hsub2(and_or(x0, 0x000f000fu, kMagic), kSub);
-        a[1] = hsub2(and_or(x1, 0x000f000fu, kMagic), kSub);
-        a[2] = hfma2(and_or(x0, 0x00f000f0u, kMagic), kInv16, kNeg72);
-        a[3] = hfma2(and_or(x1, 0x00f000f0u, kMagic), kInv16, kNeg72);
+        // byte (u_hi << 4 | u_lo), u = code + 8: (u << 4) ^ 0x80 is the int8 16 * code
+        const uint32_t x0 = w0[j], x1 = w1[j];
+        a[0] = ((x0 << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // even k of row g
+        a[1] = ((x1 << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // even k of row g + 8
+        a[2] = (x0 & 0xF0F0F0F0u) ^ 0x80808080u;         // odd k of row g
+        a[3] = (x1 & 0xF0F0F0F0u) ^ 0x80808080u;         // odd k of row g + 8
     } else {
-        // bytes biased by 128 then placed under exponent 0x64: 1024 + (code + 128); minus 1152
-        const uint32_t kHi = 0x64646464u, kSub = 0x64806480u /* 1152 */;
-        const uint32_t x0 = w0[j] ^ 0x80808080u, x1 = w1[j] ^ 0x80808080u;
-        a[0] = hsub2(prmt(x0, kHi, 0x5140u), kSub);
-        a[1] = hsub2(prmt(x1, kHi, 0x5140u), kSub);
-        a[2] = hsub2(prmt(x0, kHi, 0x7362u), kSub);
-        a[3] = hsub2(prmt(x1, kHi, 0x7362u), kSub);
+        a[0] = w0[2 * j];
+        a[1] = w1[2 * j];
+        a[2] = w0[2 * j + 1];
+        a[3] = w1[2 * j + 1];
     }
 }
 
-
-// Physical row (0..7) inside a 16-row tile of logical MMA row g (and g + 8), chosen so
-// that the shared-memory reads of one instruction hit distinct banks under the
-// 128-byte swizzle (8 lanes per phase for 16-byte reads, 16 for 8-byte, 32 for 4-byte).
+// Physical row (0..7) inside a 16-row tile of MMA row g (and g + 8), chosen so that the
+// shared-memory reads of one instruction hit distinct banks under the 128-byte swizzle
+// (8 lanes per phase for 16-byte reads, 16 for 8-byte, 32 for 4-byte).
 template <int L>
 Q4_DEVINL int row_perm(int g) {
     if constexpr (L == 16) return (g >> 1) + 4 * (g & 1);
@@ -272,109 +300,105 @@ Q4_DEVINL void lds_words(uint32_t (&dst)[L / 4], const uint8_t *p) {
     }
 }
 
-// One segment: KT k-tiles of MMAs. Z: the accumulators start from zero (first k-tiles use
-// a zero C operand instead of clearing registers).
-template <int BITS, int L, int NB, int LW, int ACC, bool Z>
-Q4_DEVINL void seg_mma(float (&c)[ACC][NB][4], const uint32_t (&w0)[L / 4], const uint32_t (&w1)[L / 4],
-                       const uint2 *fk, bool stored) {
-    constexpr int KT = (32 * L / BITS) / 16;
-#pragma unroll
-    for (int j = 0; j < KT; ++j) {
-        uint32_t af[4];
-        unpack_a<BITS, L>(af, w0, w1, j);
+// The exact group sums of one stage when its group structure is known at compile time.
+// GPS >= 1: the stage holds GPS whole groups; GPS == 0: the stage lies inside one group.
+// Every group starts with a zero-accumulator MMA; with one n8 block each group has its
+// own accumulators (independent chains), otherwise one set is flushed and reused. A flush
+// combines the two digit columns (256 * c0 + c1, exact), converts once and applies the
+// group's fp32 scale (s0p / s1p: scales of the stage's first group for rows g and g + 8).
+// frl: this lane's digits of the stage. FULL: every segment of the stage is valid;
+// otherwise the first nsl are (whole groups when GPS >= 1).
+template <int BITS, int L, int NB, int LW, int GPS, bool FULL>
+Q4_DEVINL void stage_fixed(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
+                           const uint32_t (&A1)[kTileBytes / (4 * L)][L / 4], const uint8_t *frl,
+                           const float *s0p, const float *s1p, int nsl, float (&y0)[NB], float (&y1)[NB]) {
+    constexpr int SPS = kTileBytes / (4 * L);
+    constexpr int KTI = BITS == 4 ? L / 4 : L / 8;
+    constexpr int KTS = SPS * KTI;
+    constexpr int NG = GPS > 0 ? GPS : 1;  // groups per stage
+    constexpr int IPG = KTS / NG;          // MMAs per group
+    constexpr bool PAIRED = NB <= 2;
+    constexpr int CH = NB == 1 ? NG : 1;   // accumulator sets
+    int c[CH][NB][4];
+    uint4 bq[PAIRED ? NB : 1];
+    auto flush = [&](int q, int (&cc)[NB][4]) {
+        const float s0 = s0p[q], s1 = s1p[q];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-            const uint2 bb = fk[stored ? j * NB * LW + nb * LW : 0];
-            if (Z && j < ACC)
-                mma_f16_16816_z(c[j % ACC][nb], af, bb.x, bb.y);
-            else
-                mma_f16_16816(c[j % ACC][nb], af, bb.x, bb.y);
+            const int p0 = cc[nb][0] * 256 + cc[nb][1], p1 = cc[nb][2] * 256 + cc[nb][3];
+            y0[nb] = fmaf(s0, __int2float_rn(p0), y0[nb]);
+            y1[nb] = fmaf(s1, __int2float_rn(p1), y1[nb]);
         }
-    }
-}
-
-// One stage whose GPS scale groups each lie inside it: per-group accumulator chains
-// (two alternating chains when GPS == 1), each started with a zero-C MMA, then every
-// group is flushed with its scale. FULL: all SPS segments are valid (no branches).
-template <int BITS, int L, int NB, int LW, int GPS, bool FULL>
-Q4_DEVINL void stage_groups(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
-                            const uint32_t (&A1)[kTileBytes / (4 * L)][L / 4], const uint2 *fr, bool stored,
-                            const float *sb, int pr, int g0, int nsl, float (&pa0)[NB], float (&pa1)[NB]) {
-    constexpr int KT = (32 * L / BITS) / 16;
-    constexpr int SPS = kTileBytes / (4 * L);
-    constexpr int SPG = SPS / GPS;  // segments per group
-    constexpr int CH = GPS >= 2 ? GPS : 2;
-    float cc[CH][NB][4];
+    };
 #pragma unroll
-    for (int sl = 0; sl < SPS; ++sl) {
+    for (int i = 0; i < KTS; ++i) {
+        const int sl = i / KTI, j = i % KTI, q = i / IPG, ch = CH > 1 ? q : 0;
         if (FULL || sl < nsl) {
-#pragma unroll
-            for (int j = 0; j < KT; ++j) {
-                uint32_t af[4];
-                unpack_a<BITS, L>(af, A0[sl], A1[sl], j);
-                const int q = GPS >= 2 ? sl / SPG : ((sl * KT + j) & 1);
-                const bool first = GPS >= 2 ? (sl % SPG == 0 && j == 0) : (sl * KT + j < 2);
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const uint2 bb = fr[stored ? (sl * KT + j) * NB * LW + nb * LW : 0];
-                    if (first)
-                        mma_f16_16816_z(cc[q][nb], af, bb.x, bb.y);
-                    else
-                        mma_f16_16816(cc[q][nb], af, bb.x, bb.y);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < GPS; ++q) {
-        if (FULL || q * SPG < nsl) {
-            const float s0 = sb[pr * kSG + g0 + q], s1 = sb[(pr + 8) * kSG + g0 + q];
+            uint32_t af[4];
+            unpack_a<BITS, L>(af, A0[sl], A1[sl], j);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                float h0 = cc[q][nb][0] + cc[q][nb][1], h1 = cc[q][nb][2] + cc[q][nb][3];
-                if constexpr (GPS == 1) {
-                    h0 += cc[1][nb][0] + cc[1][nb][1];
-                    h1 += cc[1][nb][2] + cc[1][nb][3];
+                uint32_t b0, b1;
+                if constexpr (PAIRED) {
+                    if ((i & 1) == 0) bq[nb] = *reinterpret_cast<const uint4 *>(frl + ((i >> 1) * NB + nb) * LW * 16);
+                    b0 = (i & 1) ? bq[nb].z : bq[nb].x;
+                    b1 = (i & 1) ? bq[nb].w : bq[nb].y;
+                } else {
+                    const uint2 bb = *reinterpret_cast<const uint2 *>(frl + (i * NB + nb) * LW * 8);
+                    b0 = bb.x;
+                    b1 = bb.y;
                 }
-                pa0[nb] = fmaf(s0, h0, pa0[nb]);
-                pa1[nb] = fmaf(s1, h1, pa1[nb]);
+                if (i % IPG == 0)
+                    mma_s8_16832_z(c[ch][nb], af, b0, b1);
+                else
+                    mma_s8_16832(c[ch][nb], af, b0, b1);
+            }
+            if constexpr (CH == 1) {
+                // one accumulator set: flush at the end of each group (GPS == 0: at the
+                // last valid segment of the stage)
+                const bool last = GPS > 0 ? (i % IPG == IPG - 1)
+                                          : (FULL ? i == KTS - 1 : (j == KTI - 1 && sl == nsl - 1));
+                if (last) flush(q, c[0]);
             }
         }
     }
+    if constexpr (CH > 1) {
+#pragma unroll
+        for (int q = 0; q < NG; ++q)
+            if (FULL || q * (SPS / NG) < nsl) flush(q, c[q]);
+    }
 }
 
-Q4_DEVINL void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// GPS > 0: every scale group lies inside one stage and a stage holds GPS whole groups
-// (the group size divides the 256-k / 128-k stage); GPS == 0: any group size that is a
-// multiple of a segment, tracked segment by segment.
-template <int BITS, int L, int NB, int LW, int GPS>
+// INK: one row of x whose digits the consumers build in shared memory (no workspace);
+// otherwise the digits come from gemv_prep through a second ring. GPS: groups per stage
+// when they divide it, 0 when the stage lies inside one group, -1 for any other group
+// size (tracked segment by segment at run time).
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16>
 __global__ void __launch_bounds__(kThreads, 2)
 gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
-    constexpr int SEGK = 32 * L / BITS;
-    constexpr int KT = SEGK / 16;
+    constexpr int SPS = kTileBytes / (4 * L);          // segments per stage
+    constexpr int KTI = BITS == 4 ? L / 4 : L / 8;     // MMAs per segment
+    constexpr int KTS = SPS * KTI;                     // MMAs per stage (8 int4, 4 int8)
     constexpr int WPT = L / 4;
-    constexpr int SPS = kTileBytes / (4 * L);  // segments per stage
-    constexpr int KTS = SPS * KT;              // k-tiles per stage
+    constexpr int STAGEK = kTileBytes * 8 / BITS;
+    constexpr bool PAIRED = NB <= 2;
+    constexpr int LW = INK ? 16 : 32;  // digit lanes stored per (MMA, n8 block)
+    static_assert(!INK || NB == 1, "in-kernel digits cover one row of x");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int nring = a.nst_ring;
-    uint8_t *slots = smem;                                  // codes: nring x 16 KB (1024-aligned)
-    uint8_t *fslots = smem + nring * kPayloadBytes;         // fragments: nring x slot_bytes
-    float *scl = reinterpret_cast<float *>(fslots + nring * a.slot_bytes);  // [2][128][kSG]
-    float *red = scl + 2 * kRowsPerCta * kSG;                               // [128][16] when CS > 1
-    uint2 *zero8 = reinterpret_cast<uint2 *>(red + (a.CS > 1 ? kRowsPerCta * 16 : 0));
-    uint64_t *full = reinterpret_cast<uint64_t *>(zero8 + 2);  // codes landed
-    uint64_t *empty = full + kMaxStages;                         // codes copied to registers
-    uint64_t *ffull = empty + kMaxStages;                        // fragments landed
-    uint64_t *fempty = ffull + kMaxStages;                       // fragments no longer read
+    uint8_t *slots = smem;                                   // codes: nring x 16 KB (1024-aligned)
+    uint8_t *fslots = smem + nring * kPayloadBytes;          // digits: ring slots, or the CTA's range
+    const int nfrag = INK ? a.stages_per_cta : nring;
+    float *scl = reinterpret_cast<float *>(fslots + nfrag * a.fslot_bytes);  // [2][128][kSG]
+    uint32_t *mx_sh = reinterpret_cast<uint32_t *>(scl + 2 * kRowsPerCta * kSG);  // [kMaxLocalBlocks]
+    uint64_t *full = reinterpret_cast<uint64_t *>(mx_sh + kMaxLocalBlocks);  // codes landed
+    uint64_t *empty = full + kMaxStages;                                  // codes copied to registers
+    uint64_t *ffull = empty + kMaxStages;                                 // digits landed
+    uint64_t *fempty = ffull + kMaxStages;                                // digits no longer read
     uint64_t *sfull = fempty + kMaxStages;
     uint64_t *sempty = sfull + 2;
+    float *red = reinterpret_cast<float *>(slots);  // [128][16] partial sums, after the main loop
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int crank = (int)(blockIdx.x % (unsigned)a.CS);
@@ -386,7 +410,6 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     const int nst = max(st_hi - st_lo, 0);
     const int seg_hi = min(st_hi * SPS, a.segs);
     const int eb_first = st_lo / a.ebs;
-    constexpr int ktile_bytes = NB * LW * 8;  // fragment bytes of one k-tile
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxStages; ++i) {
@@ -399,7 +422,6 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             mbar_init(sfull + i, 32);
             mbar_init(sempty + i, kConsumers);
         }
-        zero8[0] = zero8[1] = make_uint2(0u, 0u);
         fence_barrier_init();
     }
     __syncthreads();
@@ -412,10 +434,12 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         ng = (sg1 - 1) / a.spg - gA + 1;
     };
 
+    // 16-byte scale copies when every row of scales starts 16-byte aligned
+    const bool vec16 = (a.scales_per_row & 3) == 0 && ((uintptr_t)a.scales & 15) == 0;
     bool timed_out = false;
     if (warp == kConsumers) {
         // ---------------- producer warp ----------------
-        const uint8_t *fsrc = a.frag + (size_t)mc * (a.K / 16) * ktile_bytes;
+        const uint8_t *fsrc = a.frag + (size_t)mc * a.stages_total * a.fslot_bytes;
         const int primed = min(nst, nring);
         int slot = 0, round = 0;          // ring position, completed passes over the ring
         int eb = eb_first, eb_left = 0;   // current k-block, stages left in it
@@ -429,41 +453,50 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                 if (ebl >= 2 && !timed_out) timed_out = !mbar_wait(sempty + b, (uint32_t)(((ebl >> 1) - 1) & 1));
                 int gA, ng;
                 eb_groups(eb, gA, ng);
-                // asynchronous 4-byte copies: the producer never waits for them; rows past
-                // N copy the last row's scales (their outputs are never stored)
+                // asynchronous copies: the producer never waits for them; rows past N copy
+                // the last row's scales (their outputs are never stored). With rows of a
+                // multiple of 4 scales, whole aligned 16-byte chunks around [gA, gA + ng) are
+                // copied (a row keeps gA's offset inside its chunk, at most 12 floats).
                 float *dst = scl + b * kRowsPerCta * kSG;
-                for (int r = lane; r < kRowsPerCta; r += 32) {
-                    const int n = min(cl * kRowsPerCta + r, a.N - 1);
-                    const float *src = a.scales + (size_t)n * a.scales_per_row + gA;
-                    for (int gi = 0; gi < ng; ++gi) cp_async4(dst + r * kSG + gi, src + gi);
+                if (vec16) {
+                    const int c0 = gA & ~3, nc = (gA + ng + 3 - c0) >> 2;
+                    for (int r = lane; r < kRowsPerCta; r += 32) {
+                        const int n = min(cl * kRowsPerCta + r, a.N - 1);
+                        const float *src = a.scales + (size_t)n * a.scales_per_row + c0;
+                        for (int q = 0; q < nc; ++q) cp_async16(dst + r * kSG + 4 * q, src + 4 * q);
+                    }
+                } else {
+                    for (int r = lane; r < kRowsPerCta; r += 32) {
+                        const int n = min(cl * kRowsPerCta + r, a.N - 1);
+                        const float *src = a.scales + (size_t)n * a.scales_per_row + gA;
+                        for (int gi = 0; gi < ng; ++gi) cp_async4(dst + r * kSG + gi, src + gi);
+                    }
                 }
                 cp_async_arrive(sfull + b);
             }
             --eb_left;
-            const int ktv = min(KTS, a.K / 16 - s * KTS);
-            const uint32_t fbytes = (uint32_t)(ktv * ktile_bytes);
             if (round > 0 && !timed_out) timed_out = !mbar_wait(empty + slot, (uint32_t)((round - 1) & 1));
             if (lane == 0 && !timed_out) {
                 mbar_arrive_expect_tx(full + slot, kPayloadBytes);
                 tma_load_2d(slots + slot * kPayloadBytes, &tmap, full + slot, s * kTileBytes, cl * kRowsPerCta);
             }
-            if (ks >= primed) {
-                if (!timed_out) timed_out = !mbar_wait(fempty + slot, (uint32_t)((round - 1) & 1));
-                if (lane == 0 && !timed_out) {
-                    mbar_arrive_expect_tx(ffull + slot, fbytes);
-                    bulk_copy_g2s(fslots + slot * a.slot_bytes, fsrc + (size_t)s * KTS * ktile_bytes, fbytes,
-                                  ffull + slot);
+            if constexpr (!INK) {
+                const uint32_t fb = (uint32_t)a.fslot_bytes;
+                if (ks >= primed) {
+                    if (!timed_out) timed_out = !mbar_wait(fempty + slot, (uint32_t)((round - 1) & 1));
+                    if (lane == 0 && !timed_out) {
+                        mbar_arrive_expect_tx(ffull + slot, fb);
+                        bulk_copy_g2s(fslots + slot * fb, fsrc + (size_t)s * fb, fb, ffull + slot);
+                    }
                 }
-            }
-            if (ks == primed - 1) {
-                // the ring is primed with codes; the fragments come from gemv_prep
-                grid_dep_wait();
-                if (lane == 0 && !timed_out) {
-                    for (int q = 0; q < primed; ++q) {
-                        const int sq = st_lo + q;
-                        const uint32_t fq = (uint32_t)(min(KTS, a.K / 16 - sq * KTS) * ktile_bytes);
-                        mbar_arrive_expect_tx(ffull + q, fq);
-                        bulk_copy_g2s(fslots + q * a.slot_bytes, fsrc + (size_t)sq * KTS * ktile_bytes, fq, ffull + q);
+                if (ks == primed - 1) {
+                    // the ring is primed with codes; the digits come from gemv_prep
+                    grid_dep_wait();
+                    if (lane == 0 && !timed_out) {
+                        for (int q = 0; q < primed; ++q) {
+                            mbar_arrive_expect_tx(ffull + q, fb);
+                            bulk_copy_g2s(fslots + q * fb, fsrc + (size_t)(st_lo + q) * fb, fb, ffull + q);
+                        }
                     }
                 }
             }
@@ -471,8 +504,61 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         }
     } else {
         // ---------------- consumers ----------------
-        grid_dep_wait();  // the exponents are read from global memory
         const int g = lane >> 2, t = lane & 3;
+        const int ct = threadIdx.x;  // 0..255
+        if constexpr (INK) {
+            // digits of this CTA's K range of the single activation row, built while the
+            // first payload tiles are in flight
+            const int nlb = nst > 0 ? (st_hi - 1) / a.ebs - eb_first + 1 : 0;
+            for (int i = ct; i < nlb; i += kConsumerThreads) mx_sh[i] = 0;
+            named_barrier_sync(1, kConsumerThreads);
+            const int k_lo = st_lo * STAGEK, k_hi = min(st_hi * STAGEK, a.K);
+            const int nu = max(k_hi - k_lo, 0) / 8;
+            constexpr int R = kFragCap / 4 / 8 / kConsumerThreads;  // units per thread (4)
+            float v[R][8];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int u = ct + kConsumerThreads * r;
+                if (u < nu) {
+                    load_x8<XBF16>(a.x, (int64_t)k_lo + 8 * u, v[r]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[r][q] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                // a warp's 32 units are 256 consecutive k: at most two k-blocks
+                const int u = ct + kConsumerThreads * r;
+                const int lb = u < nu ? (st_lo + (8 * u) / STAGEK) / a.ebs - eb_first : -1;
+                const uint32_t m = absmax8(v[r]);
+                const int lbA = __shfl_sync(0xffffffffu, lb, 0);
+                const uint32_t mA = __reduce_max_sync(0xffffffffu, lb == lbA ? m : 0u);
+                const uint32_t mB = __reduce_max_sync(0xffffffffu, (lb >= 0 && lb != lbA) ? m : 0u);
+                if (lane == 0 && lbA >= 0) {
+                    atomicMax(mx_sh + lbA, mA);
+                    if (mB) atomicMax(mx_sh + lbA + 1, mB);
+                }
+            }
+            named_barrier_sync(1, kConsumerThreads);
+            uint2 *fbase = reinterpret_cast<uint2 *>(fslots);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int u = ct + kConsumerThreads * r;
+                if (u < nu) {
+                    const int ls = (8 * u) / STAGEK;  // local stage
+                    const int lb = (st_lo + ls) / a.ebs - eb_first;
+                    const int sh = 30 - block_exp(mx_sh[lb]);
+                    const int e1 = min(max(sh, -126), 127);
+                    const float f1 = pow2(e1), f2 = pow2(min(max(sh - e1, -126), 127));
+                    frag_unit<BITS, L>(fbase + (size_t)ls * (a.fslot_bytes / 8), 8 * u - ls * STAGEK, 0, v[r], f1,
+                                       f2, 1, LW, true);
+                }
+            }
+            named_barrier_sync(1, kConsumerThreads);
+        } else {
+            grid_dep_wait();  // the exponents are read from global memory
+        }
         const int pr = 16 * warp + row_perm<L>(g);  // physical row of MMA row g in the CTA
         const int row0 = cl * kRowsPerCta + pr, row1 = row0 + 8;
         const bool ok0 = row0 < a.N, ok1 = row1 < a.N;
@@ -482,44 +568,49 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             const int off = sl * 4 * L + t * L;
             aoff[sl] = pr * kTileBytes + (((off >> 4) ^ (pr & 7)) << 4) + (off & 15);
         }
-        const bool stored = lane < LW;  // lanes beyond the stored width read zeros
-        constexpr int ACC = NB == 1 ? 2 : 1;  // two accumulator chains when there is one column block
-        float acc0[NB], acc1[NB], pa0[NB], pa1[NB], c[ACC][NB][4];
-        int ecur[NB];
+        const int fl = lane & (LW - 1);  // lanes past the stored width repeat lanes (their columns are unused)
+        // fold exponent of this lane's columns: 2^(E-30), 2^-4 for the int4 factor 16,
+        // 2^16 for the high digit pair (t even)
+        const int fadj = -30 - (BITS == 4 ? 4 : 0) + ((t & 1) == 0 ? 16 : 0);
+        int c[NB][4];
+        float y0[NB], y1[NB], acc0[NB], acc1[NB];
+        int fe[NB], enext[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-            acc0[nb] = acc1[nb] = pa0[nb] = pa1[nb] = 0.f;
-            ecur[nb] = 0;
+            c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0;
+            y0[nb] = y1[nb] = acc0[nb] = acc1[nb] = 0.f;
+            fe[nb] = enext[nb] = 0;
+        }
+        auto load_exps = [&](int eb) {
 #pragma unroll
-            for (int q = 0; q < ACC; ++q) c[q][nb][0] = c[q][nb][1] = c[q][nb][2] = c[q][nb][3] = 0.f;
+            for (int nb = 0; nb < NB; ++nb) {
+                const int ml = 2 * nb + (t >> 1);
+                enext[nb] = ml < mcnt ? a.ebexp[(int64_t)(mc * 16 + ml) * a.n_eb + eb] : 0;
+            }
+        };
+        if constexpr (!INK) {
+            if (nst > 0) load_exps(eb_first);
         }
         int lg = (st_lo * SPS) / a.spg;                 // group of the next segment
         int crem = a.spg - (st_lo * SPS - lg * a.spg);  // segments left in that group
         int gA = 0, ng = 0, b = 0;
-        bool fresh = true;                              // the accumulators hold nothing yet
         const float *sb = scl;
-        auto flush = [&]() {
-            const float s0 = sb[pr * kSG + (lg - gA)], s1 = sb[(pr + 8) * kSG + (lg - gA)];
+        auto flush = [&](int q) {  // a group (or a stage) ends: scale its exact sums
+            const float s0 = sb[pr * kSG + q], s1 = sb[(pr + 8) * kSG + q];
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                float h0 = c[0][nb][0] + c[0][nb][1], h1 = c[0][nb][2] + c[0][nb][3];
-                if constexpr (ACC == 2) {
-                    h0 += c[1][nb][0] + c[1][nb][1];
-                    h1 += c[1][nb][2] + c[1][nb][3];
-                }
-                pa0[nb] = fmaf(s0, h0, pa0[nb]);
-                pa1[nb] = fmaf(s1, h1, pa1[nb]);
-#pragma unroll
-                for (int q = 0; q < ACC; ++q) c[q][nb][0] = c[q][nb][1] = c[q][nb][2] = c[q][nb][3] = 0.f;
+                const int p0 = c[nb][0] * 256 + c[nb][1], p1 = c[nb][2] * 256 + c[nb][3];
+                y0[nb] = fmaf(s0, __int2float_rn(p0), y0[nb]);
+                y1[nb] = fmaf(s1, __int2float_rn(p1), y1[nb]);
+                c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0;
             }
-            fresh = true;
         };
-        auto fold = [&]() {  // end of a k-block: apply its 2^e exactly
+        auto fold = [&]() {  // end of a k-block: apply its power of two exactly
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                acc0[nb] += ldexpf(pa0[nb], ecur[nb]);
-                acc1[nb] += ldexpf(pa1[nb], ecur[nb]);
-                pa0[nb] = pa1[nb] = 0.f;
+                acc0[nb] += scale2(y0[nb], fe[nb]);
+                acc1[nb] += scale2(y1[nb], fe[nb]);
+                y0[nb] = y1[nb] = 0.f;
             }
         };
         int slot = 0, round = 0;
@@ -528,7 +619,6 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             const int s = st_lo + ks;
             if (eb_left == 0) {
                 if (ks > 0) {
-                    if (!fresh) flush();  // a group cut by the k-block boundary
                     fold();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(sempty + b);
@@ -538,11 +628,13 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                 const int ebl = eb - eb_first;
                 b = ebl & 1;
                 eb_groups(eb, gA, ng);
-                sb = scl + b * kRowsPerCta * kSG;
+                sb = scl + b * kRowsPerCta * kSG + (vec16 ? (gA & 3) : 0);
+                if constexpr (INK) {
+                    fe[0] = block_exp(mx_sh[ebl]) + fadj;
+                } else {
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int ml = nb * 4 + t;
-                    ecur[nb] = ml < mcnt ? a.ebexp[(int64_t)(mc * 16 + ml) * a.n_eb + eb] : 0;
+                    for (int nb = 0; nb < NB; ++nb) fe[nb] = enext[nb] + fadj;
+                    if ((eb + 1) * a.ebs < st_hi) load_exps(eb + 1);  // one block ahead
                 }
                 if (!timed_out) timed_out = !mbar_wait(sfull + b, (uint32_t)((ebl >> 1) & 1));
             }
@@ -558,57 +650,95 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + slot);  // the codes now live in registers: refill
-            if (!timed_out) timed_out = !mbar_wait(ffull + slot, (uint32_t)(round & 1));
-            const uint2 *fr = stored ? reinterpret_cast<const uint2 *>(fslots + slot * a.slot_bytes) + lane : zero8;
-            if constexpr (GPS > 0) {
-                // whole groups inside the stage: one accumulator chain per group (two
-                // alternating chains when the stage is one group), all flushed at its end.
-                // A full stage is one branch-free block, so the chains interleave.
-                const int g0 = s * GPS - gA;  // this stage's first group, relative to the k-block
-                if (nsl == SPS)
-                    stage_groups<BITS, L, NB, LW, GPS, true>(A0, A1, fr, stored, sb, pr, g0, SPS, pa0, pa1);
-                else
-                    stage_groups<BITS, L, NB, LW, GPS, false>(A0, A1, fr, stored, sb, pr, g0, nsl, pa0, pa1);
+            const uint8_t *fr;
+            if constexpr (INK) {
+                fr = fslots + ks * a.fslot_bytes;
             } else {
+                if (!timed_out) timed_out = !mbar_wait(ffull + slot, (uint32_t)(round & 1));
+                fr = fslots + slot * a.fslot_bytes;
+            }
+            if constexpr (GPS >= 0) {
+                const int qb = (GPS > 0 ? s * GPS : (s * SPS) / a.spg) - gA;  // first group, in the k-block
+                const float *s0p = sb + pr * kSG + qb, *s1p = s0p + 8 * kSG;
+                const uint8_t *frl = fr + fl * (PAIRED ? 16 : 8);
+                if (nsl == SPS)
+                    stage_fixed<BITS, L, NB, LW, GPS, true>(A0, A1, frl, s0p, s1p, nsl, y0, y1);
+                else
+                    stage_fixed<BITS, L, NB, LW, GPS, false>(A0, A1, frl, s0p, s1p, nsl, y0, y1);
+            } else {
+                uint4 bq[PAIRED ? NB : 1];
 #pragma unroll
-                for (int sl = 0; sl < SPS; ++sl) {
+                for (int i = 0; i < KTS; ++i) {
+                    const int sl = i / KTI, j = i % KTI;
                     if (sl < nsl) {
-                        const uint2 *fk = fr + (stored ? sl * KT * NB * LW : 0);
-                        seg_mma<BITS, L, NB, LW, ACC, false>(c, A0[sl], A1[sl], fk, stored);
-                        fresh = false;
-                        if (--crem == 0) {  // this segment ends a scale group
-                            flush();
-                            crem = a.spg;
-                            ++lg;
+                        uint32_t af[4];
+                        unpack_a<BITS, L>(af, A0[sl], A1[sl], j);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            uint32_t b0, b1;
+                            if constexpr (PAIRED) {
+                                if ((i & 1) == 0)
+                                    bq[nb] = *reinterpret_cast<const uint4 *>(
+                                        fr + 8 * (size_t)frag_idx(i, nb, fl, NB, LW, true));
+                                b0 = (i & 1) ? bq[nb].z : bq[nb].x;
+                                b1 = (i & 1) ? bq[nb].w : bq[nb].y;
+                            } else {
+                                const uint2 bb = *reinterpret_cast<const uint2 *>(
+                                    fr + 8 * (size_t)frag_idx(i, nb, fl, NB, LW, false));
+                                b0 = bb.x;
+                                b1 = bb.y;
+                            }
+                            mma_s8_16832(c[nb], af, b0, b1);
+                        }
+                        if (j == KTI - 1) {  // end of a segment
+                            const bool gend = --crem == 0;
+                            if (gend || sl == nsl - 1) {
+                                flush(lg - gA);
+                                if (gend) {
+                                    ++lg;
+                                    crem = a.spg;
+                                }
+                            }
                         }
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(fempty + slot);
+            if constexpr (!INK) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fempty + slot);
+            }
             if (++slot == nring) { slot = 0; ++round; }
         }
-        if (nst > 0) {
-            if (!fresh) flush();
-            fold();
+        if (nst > 0) fold();
+        // high + low digit halves: lane t (even) takes lane t + 1's half
+        float tot0[NB], tot1[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            tot0[nb] = acc0[nb] + __shfl_xor_sync(0xffffffffu, acc0[nb], 1);
+            tot1[nb] = acc1[nb] + __shfl_xor_sync(0xffffffffu, acc1[nb], 1);
         }
         if (a.CS == 1) {
+            if ((t & 1) == 0) {
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int ml = nb * 4 + t;
-                if (ml < mcnt) {
-                    float *yr = a.y + (int64_t)(mc * 16 + ml) * a.N;
-                    if (ok0) yr[row0] = acc0[nb];
-                    if (ok1) yr[row1] = acc1[nb];
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int ml = 2 * nb + (t >> 1);
+                    if (ml < mcnt) {
+                        float *yr = a.y + (int64_t)(mc * 16 + ml) * a.N;
+                        if (ok0) yr[row0] = tot0[nb];
+                        if (ok1) yr[row1] = tot1[nb];
+                    }
                 }
             }
         } else {
+            named_barrier_sync(1, kConsumerThreads);  // every warp is done with the ring
+            if ((t & 1) == 0) {
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int ml = nb * 4 + t;
-                if (ml < mcnt) {
-                    red[pr * 16 + ml] = acc0[nb];
-                    red[(pr + 8) * 16 + ml] = acc1[nb];
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int ml = 2 * nb + (t >> 1);
+                    if (ml < mcnt) {
+                        red[pr * 16 + ml] = tot0[nb];
+                        red[(pr + 8) * 16 + ml] = tot1[nb];
+                    }
                 }
             }
         }
@@ -653,16 +783,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int BITS, int L, int NB, int LW, int GPS>
-cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool xbf16,
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16>
+cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
                          cudaStream_t st) {
-    if (xbf16)
-        gemv_prep<BITS, L, NB, true><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
-    else
-        gemv_prep<BITS, L, NB, false><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    auto kern = gemv_stream<BITS, L, NB, LW, GPS>;
+    cudaError_t err;
+    if constexpr (!INK) {
+        if (x_bf16)
+            gemv_prep<BITS, L, true><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
+        else
+            gemv_prep<BITS, L, false><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16>;
     const size_t smem = pl.smem_bytes;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
@@ -679,47 +812,39 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = INK ? 1 : 2;  // the in-kernel path reads x at once: no early start
     return cudaLaunchKernelEx(&cfg, kern, a, tm);
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
-                          cudaStream_t st, int64_t group) {
-    // groups per 128-byte stage when the group size divides the stage, else 0
-    const int stagek = kTileBytes * 8 / pl.bits;
-    const int gps = (stagek % group == 0) ? (int)(stagek / group) : 0;
-#define Q4_LW(B, LL, NBB, G)                                                                       \
-    if constexpr (NBB == 1) {                                                                      \
-        if (pl.lw == 8) return launch_typed<B, LL, NBB, 8, G>(pl, a, tm, x_bf16, st);             \
-    }                                                                                              \
-    return launch_typed<B, LL, NBB, 32, G>(pl, a, tm, x_bf16, st);
-// per-group chains cost registers: kept for one column block, or two with at most 2 groups
-#define Q4_GPS(B, LL, NBB, G1, G2)                                                                 \
-    if (pl.bits == B && pl.L == LL && pl.NB == NBB) {                                              \
-        if constexpr (NBB == 1 || (NBB == 2 && G1 <= 2)) {                                         \
-            if (gps == G1) { Q4_LW(B, LL, NBB, G1) }                                               \
-        }                                                                                          \
-        if constexpr (G2 > 0 && NBB <= 2) {                                                        \
-            if (gps == G2) { Q4_LW(B, LL, NBB, G2) }                                               \
-        }                                                                                          \
-        Q4_LW(B, LL, NBB, 0)                                                                       \
+                          cudaStream_t st) {
+#define Q4_INK(B, LL, G)                                                                         \
+    if (pl.bits == B && pl.L == LL && pl.gps == G)                                               \
+        return x_bf16 ? launch_typed<B, LL, 1, G, true, true>(pl, a, tm, true, st)               \
+                      : launch_typed<B, LL, 1, G, true, false>(pl, a, tm, false, st);
+#define Q4_STAGED(B, LL, G)                                                                      \
+    if (pl.bits == B && pl.L == LL && pl.gps == G) {                                             \
+        switch (pl.NB) {                                                                         \
+            case 1: return launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, st);       \
+            case 2: return launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, st);       \
+            case 4: return launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, st);       \
+            default: return launch_typed<B, LL, 8, G, false, false>(pl, a, tm, x_bf16, st);      \
+        }                                                                                        \
     }
-#define Q4_GEMV(B, LL, NBB) Q4_GPS(B, LL, NBB, (LL == 16 ? 2 : LL == 8 ? 4 : 8), (LL == 16 ? 1 : 0))
-    Q4_GEMV(4, 16, 1) Q4_GEMV(4, 16, 2) Q4_GEMV(4, 16, 4)
-    Q4_GEMV(4, 8, 1) Q4_GEMV(4, 8, 2) Q4_GEMV(4, 8, 4)
-    Q4_GEMV(4, 4, 1) Q4_GEMV(4, 4, 2) Q4_GEMV(4, 4, 4)
-    Q4_GEMV(8, 16, 1) Q4_GEMV(8, 16, 2) Q4_GEMV(8, 16, 4)
-    Q4_GEMV(8, 8, 1) Q4_GEMV(8, 8, 2) Q4_GEMV(8, 8, 4)
-    Q4_GEMV(8, 4, 1) Q4_GEMV(8, 4, 2) Q4_GEMV(8, 4, 4)
-#undef Q4_GEMV
-#undef Q4_GPS
-#undef Q4_LW
+#define Q4_ALL(M)                                                                                \
+    M(4, 16, 2) M(4, 16, 0) M(4, 8, 4) M(4, 4, 8) M(4, 4, -1) M(8, 16, 2) M(8, 16, 0) M(8, 8, 4) M(8, 8, -1)
+    if (pl.ink) {
+        Q4_ALL(Q4_INK)
+    } else {
+        Q4_ALL(Q4_STAGED)
+    }
+#undef Q4_ALL
+#undef Q4_STAGED
+#undef Q4_INK
     return cudaErrorInvalidValue;
 }
-
-
 
 }  // namespace
 
@@ -727,27 +852,36 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
     GemvPlan p = {};
     p.bits = bits;
     if (K % 32 != 0 || group <= 0 || K % group != 0) return false;
+    // a segment (4 lanes x L bytes of a row) must lie inside one scale group
     if (bits == 4)
         p.L = group % 128 == 0 ? 16 : group % 64 == 0 ? 8 : group % 32 == 0 ? 4 : 0;
     else
-        p.L = group % 64 == 0 ? 16 : group % 32 == 0 ? 8 : group % 16 == 0 ? 4 : 0;
+        p.L = group % 64 == 0 ? 16 : group % 32 == 0 ? 8 : 0;
     if (!p.L) return false;
+    // groups per 128-byte stage when they divide it, 0 when the stage lies inside one
+    // group, -1 otherwise (then the narrowest segments, which always fit in a group)
+    {
+        const int64_t sk = kTileBytes * 8 / bits;
+        p.gps = sk % group == 0 ? (int)(sk / group) : group % sk == 0 ? 0 : -1;
+        if (p.gps == 1) p.gps = 0;  // one group per stage: the same as a stage inside a group
+        if (p.gps < 0) p.L = bits == 4 ? 4 : 8;
+    }
     if (K > ((int64_t)1 << 30) || N > ((int64_t)1 << 30) || M > ((int64_t)1 << 20)) return false;
     p.segk = 32 * p.L / bits;
     p.segs = (int)(K / p.segk);
     p.spg = (int)(group / p.segk);
     p.nmc = (int)((M + 15) / 16);
     const int mc0 = (int)(M < 16 ? M : 16);
-    p.NB = mc0 > 8 ? 4 : mc0 > 4 ? 2 : 1;
-    p.lw = (M == 1) ? 8 : 32;  // one row of x: only lanes 0..7 carry fragments
-    p.T = (int)((N + 15) / 16);
+    const int nbm = (mc0 + 1) / 2;  // n8 blocks needed: two rows of x (4 digits each) per block
+    p.NB = nbm <= 1 ? 1 : nbm <= 2 ? 2 : nbm <= 4 ? 4 : 8;
+    p.paired = p.NB <= 2;
     p.clusters = (int)((N + kRowsPerCta - 1) / kRowsPerCta);
     const int64_t rowbytes = K * bits / 8;
     p.stages_total = (int)((rowbytes + kTileBytes - 1) / kTileBytes);
     const int stagek = kTileBytes * 8 / bits;
-    // k-block: <= 16 scale groups and <= 2048 k, in whole stages
-    int64_t ebs = 16 * group / stagek;
-    if (ebs > 2048 / stagek) ebs = 2048 / stagek;
+    // k-block: about kGroupsPerBlock scale groups and at most kBlockK k, in whole stages
+    int64_t ebs = kGroupsPerBlock * group / stagek;
+    if (ebs > kBlockK / stagek) ebs = kBlockK / stagek;
     if (ebs < 1) ebs = 1;
     p.ebs = (int)ebs;
     p.n_eb = (p.stages_total + p.ebs - 1) / p.ebs;
@@ -759,19 +893,32 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
     if (cs > p.stages_total / 2) cs = p.stages_total / 2;
     p.CS = cs < 1 ? 1 : (int)cs;
     p.stages_per_cta = (p.stages_total + p.CS - 1) / p.CS;
-    // ring stage = 16 KB of codes + the stage's fragments (slot_bytes, 16-aligned)
-    const int kts = kTileBytes / (4 * p.L) * (p.segk / 16);
-    p.slot_bytes = (int)align_up((size_t)kts * p.NB * p.lw * 8, 16);
-    const size_t fixed = 1024 + 2 * (size_t)kRowsPerCta * kSG * 4 + (p.CS > 1 ? (size_t)kRowsPerCta * 16 * 4 : 0) +
-                         16 + (4 * kMaxStages + 4) * 8;
-    const size_t budget = 111 * 1024;  // two CTAs per SM
-    int nr = (int)((budget - fixed) / (kPayloadBytes + p.slot_bytes));
-    p.nst_ring = nr > kMaxStages ? kMaxStages : nr < 2 ? 2 : nr;
-    p.smem_bytes = fixed + (size_t)p.nst_ring * (kPayloadBytes + p.slot_bytes);
-    // workspace: fragments [mc][k-tile][nb][lw] x 8 bytes, then exponents [mc*16][n_eb]
-    p.off_frag = 0;
-    p.off_exp = align_up((size_t)p.nmc * (K / 16) * p.NB * p.lw * 8, 256);
-    p.bytes = align_up(p.off_exp + (size_t)p.nmc * 16 * p.n_eb * 4, 256);
+    const int kts = bits == 4 ? 8 : 4;  // MMAs per stage
+    // one row of x: 16 digit lanes, built on chip when the CTA's K range fits
+    p.ink = M == 1 && (int64_t)p.stages_per_cta * kts * 16 * 8 <= kFragCap;
+    p.lw = p.ink ? 16 : 32;
+    p.fslot_bytes = kts * p.NB * p.lw * 8;
+    const size_t fixed = 1024 + 2 * (size_t)kRowsPerCta * kSG * 4 + kMaxLocalBlocks * 4 + (4 * kMaxStages + 4) * 8;
+    int nr;
+    if (p.ink) {
+        const size_t frag = (size_t)p.stages_per_cta * p.fslot_bytes;
+        nr = (int)((kSmemBudget - fixed - frag) / kPayloadBytes);
+        p.nst_ring = nr > kMaxStages ? kMaxStages : nr < 2 ? 2 : nr;
+        p.smem_bytes = fixed + frag + (size_t)p.nst_ring * kPayloadBytes;
+    } else {
+        nr = (int)((kSmemBudget - fixed) / (kPayloadBytes + p.fslot_bytes));
+        p.nst_ring = nr > kMaxStages ? kMaxStages : nr < 2 ? 2 : nr;
+        p.smem_bytes = fixed + (size_t)p.nst_ring * (kPayloadBytes + p.fslot_bytes);
+    }
+    static_assert(kRedBytes <= 2 * kPayloadBytes, "partial sums fit in the ring");
+    // workspace (several rows of x): digits [mc][stage][fslot_bytes], then exponents [mc*16][n_eb]
+    if (p.ink) {
+        p.off_frag = p.off_exp = p.bytes = 0;
+    } else {
+        p.off_frag = 0;
+        p.off_exp = align_up((size_t)p.nmc * p.stages_total * p.fslot_bytes, 256);
+        p.bytes = align_up(p.off_exp + (size_t)p.nmc * 16 * p.n_eb * 4, 256);
+    }
     *pl = p;
     return true;
 }
@@ -797,8 +944,8 @@ cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t 
     a.x = x;
     a.y = y;
     a.status = status;
-    a.frag = reinterpret_cast<const uint8_t *>(w + pl.off_frag);
-    a.ebexp = reinterpret_cast<int *>(w + pl.off_exp);
+    a.frag = w ? reinterpret_cast<uint8_t *>(w + pl.off_frag) : nullptr;
+    a.ebexp = w ? reinterpret_cast<int *>(w + pl.off_exp) : nullptr;
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
@@ -811,9 +958,11 @@ cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t 
     a.ebs = pl.ebs;
     a.n_eb = pl.n_eb;
     a.lw = pl.lw;
+    a.NB = pl.NB;
+    a.paired = pl.paired;
     a.nst_ring = pl.nst_ring;
-    a.slot_bytes = pl.slot_bytes;
-    return dispatch_gemv(pl, a, tm, x_bf16, st, group);
+    a.fslot_bytes = pl.fslot_bytes;
+    return dispatch_gemv(pl, a, tm, x_bf16, st);
 }
 
 }  // namespace q4

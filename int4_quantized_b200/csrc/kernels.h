@@ -16,25 +16,27 @@ cudaError_t launch_qdequant(const uint8_t *payload, const float *scales, int64_t
 
 // ---- decode GEMV --------------------------------------------------------------------
 // Plan of one GEMV call: how K is cut into segments (one 128/64/32-bit load per lane per
-// weight row), how a thread-block cluster splits K, and how much x is staged at a time.
+// weight row), how a thread-block cluster splits K, and where the activation digits live.
 struct GemvPlan {
     int bits, L;        // L = bytes each lane reads per weight row per segment (16, 8 or 4)
     int segk;           // k per segment = 32 * L / bits
     int segs;           // segments per row = K / segk
     int spg;            // segments per scale group = group / segk
-    int NB;             // n8 blocks of activation columns per 16-row chunk of x (1, 2 or 4)
-    int lw;             // fragment lanes stored per (k-tile, n8 block)
-    int T;              // 16-row tiles of W = ceil(N / 16)
+    int gps;            // groups per stage (divides it), 0 (stage inside a group) or -1
+    int NB;             // n8 blocks of MMA columns per 16-row chunk of x (1, 2, 4 or 8)
+    int lw;             // digit lanes stored per (MMA, n8 block): 16 on chip, 32 in the workspace
+    int paired;         // digits of two consecutive MMAs interleaved
     int clusters;       // CTAs along N = ceil(N / 128)
     int CS;             // CTAs per cluster = splits of K (1..8)
     int stages_total;   // 128-byte tiles per weight row
     int stages_per_cta; // tiles per CTA's K range
     int ebs, n_eb;      // tiles per k-block (exponent and scale block), k-blocks per row
     int nst_ring;       // ring depth
-    int slot_bytes;     // bytes of one ring slot
+    int fslot_bytes;    // digit bytes of one stage
+    int ink;            // one row of x: digits built in shared memory, no workspace
     int nmc;            // 16-row chunks of x = ceil(M / 16)
     size_t smem_bytes;  // dynamic shared memory per CTA
-    size_t off_frag, off_exp, bytes;  // workspace layout and size
+    size_t off_frag, off_exp, bytes;  // workspace layout and size (0 when ink)
 };
 
 // Returns false when this GEMV does not cover (bits, group, K).

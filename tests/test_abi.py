@@ -80,7 +80,8 @@ def test_qpack_validation(q4, rows, cols, bits, group, ptr_ok, expect):
     (1, 64, 96, 4, 64, 0, 2),       # group does not divide K
     (1, 64, 48, 4, 48, 0, 2),       # K % 32
     (1, 64, 128, 4, 16, 0, 2),      # int4 group % 32
-    (1, 64, 128, 8, 8, 0, 2),       # int8 group % 16
+    (1, 64, 128, 8, 8, 0, 2),       # int8 group % 32
+    (1, 64, 128, 8, 16, 0, 2),      # int8 group % 32
     (-1, 64, 128, 4, 128, 0, 1),    # negative M
 ])
 def test_qgemm_validation(q4, M, N, K, bits, group, xt, expect):
