@@ -133,6 +133,7 @@ size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64
                                 q4_xdtype xt) {
     q4::GemvPlan pl;
     if (plan_qgemm(M, N, K, bits, group, xt, &pl) != Q4_OK) return 0;
+    if (q4::prefill_supported(M, N, K, bits, group, xt == Q4_X_BF16)) return 0;
     return pl.bytes;
 }
 
@@ -145,6 +146,11 @@ q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
     if (M == 0 || N == 0) return Q4_OK;
     if (!x || !payload || !scales || !y) return Q4_ERR_ARG;
     if ((uintptr_t)payload % 16 || (uintptr_t)x % 16) return Q4_ERR_UNSUPPORTED;
+    if (q4::prefill_supported(M, N, K, bits, group, xt == Q4_X_BF16)) {
+        cudaError_t e = q4::launch_prefill(x, M, payload, scales, N, K, bits, group, y, status_word,
+                                           device_sms(), as_stream(stream));
+        return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    }
     if ((uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return Q4_ERR_WORKSPACE;
     cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,

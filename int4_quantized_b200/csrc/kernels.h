@@ -46,4 +46,11 @@ cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t 
                         const uint8_t *payload, const float *scales, int64_t N, int64_t K,
                         int64_t group, float *y, void *ws, uint32_t *status, cudaStream_t st);
 
+// ---- prefill GEMM (tcgen05) ----------------------------------------------------------
+// bf16 x with M >= 64, K and group multiples of 64: the tensor-memory GEMM of prefill.cu.
+bool prefill_supported(int64_t M, int64_t N, int64_t K, int bits, int64_t group, bool x_bf16);
+cudaError_t launch_prefill(const void *x, int64_t M, const uint8_t *payload, const float *scales, int64_t N,
+                           int64_t K, int bits, int64_t group, float *y, uint32_t *status, int sms,
+                           cudaStream_t st);
+
 }  // namespace q4
