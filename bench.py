@@ -66,6 +66,24 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time: every rank passes its own device time; with one process
+    (no process group) it is returned unchanged."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: every rank moves bytes_per_step per step (weak scaling) in ms."""
+    return bytes_per_step * steps * world / (ms / 1e3) / 1e9
+
+
 def step_bytes(N, K, formats, Ms):
     """Algorithmic bytes per kernel of one step: {key: bytes}."""
     out = {}
@@ -358,11 +376,8 @@ def run_ours(args):
     if ClockSampler.rejected(clocks):
         ms, clocks = timed(args.steps)  # measured once more, as the rules ask
         clocks["remeasured"] = True
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = bytes_per_step * args.steps * world / (ms / 1e3) / 1e9
+    ms = max_over_ranks(ms, dev)
+    value = job_throughput(bytes_per_step, args.steps, world, ms)
 
     # per-kernel device time: graphs of ROT launches of one kernel kind, same buffers
     per_kernel = {}
