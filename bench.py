@@ -321,7 +321,9 @@ def run_ours(args):
     def key(kind, f, M):
         return f"qpack_int{f[0]}_g{f[1]}" if kind == "qpack" else f"gemv_int{f[0]}_g{f[1]}_M{M}"
 
-    launches_per_step = sum(1 if k == "qpack" else 2 for k, _, _ in plan)
+    # qpack: one kernel; qgemm: the stream kernel, plus gemv_prep when it needs a workspace
+    launches_per_step = sum(1 if k == "qpack" else (2 if q4.qgemm_workspace_bytes(M, N, K, f[0], f[1]) else 1)
+                            for k, f, M in plan)
     kbytes = step_bytes(N, K, formats, Ms)
     bytes_per_step = sum(kbytes.values())
 
