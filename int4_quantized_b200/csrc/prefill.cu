@@ -39,13 +39,13 @@ constexpr int kBN = 256;          // activation rows per tile (MMA N)
 constexpr int kBK = 64;           // k per step: one 128-byte swizzle row of bf16
 constexpr int kStages = 4;        // x + payload ring
 constexpr int kAStages = 3;       // dequantized A ring
-constexpr int kThreads = 384;
+constexpr int kThreads = 384;     // grouped scales: TMA, MMA, 2 dequantizing, 8 epilogue warps
+constexpr int kThreadsPC = 320;   // one scale per output channel: TMA, MMA, 4 + 4
 constexpr int kXBytes = kBN * kBK * 2;        // 32 KB
 constexpr int kABytes = kBM * kBK * 2;        // 16 KB
 constexpr int kPBytesMax = kBM * kBK;         // 8 KB (int8); int4 uses half
 constexpr int kTmemCols = 512;                // two D buffers of 256 columns
-constexpr int kEpiWarps = 8;
-constexpr int kDqThreads = 64;
+
 
 struct PrefillArgs {
     const float *scales;
@@ -56,7 +56,30 @@ struct PrefillArgs {
     int kpg;              // k-steps per scale group
     int ksteps;           // K / kBK
     int tiles_n, tiles;   // output tiles: (N / 128) x (M / 256), n fastest
+    int full_items;       // items that are whole tiles (a multiple of the grid)
+    int split;            // the remaining tiles are cut into `split` narrower items (1, 2 or 4)
+    int items;            // full_items + (tiles - full_items) * split
 };
+
+// Work item j (CTA j % grid takes it): output rows [n0, n0 + 128) x activation rows
+// [m0, m0 + width). Whole tiles fill the complete rounds of the grid; the tiles of the
+// last, partial round are cut along the activation rows so that round is shorter.
+struct Item {
+    int n0, m0, width;
+};
+Q4_DEVINL Item item_of(const PrefillArgs &a, int j) {
+    Item it;
+    int t = j, part = 0;
+    it.width = kBN;
+    if (j >= a.full_items) {
+        t = a.full_items + (j - a.full_items) / a.split;
+        part = (j - a.full_items) % a.split;
+        it.width = kBN / a.split;
+    }
+    it.n0 = (t % a.tiles_n) * kBM;
+    it.m0 = (t / a.tiles_n) * kBN + part * it.width;
+    return it;
+}
 
 // ---- tcgen05 helpers -------------------------------------------------------------------
 Q4_DEVINL void tmem_alloc(uint32_t *dst, uint32_t ncols) {
@@ -145,11 +168,17 @@ Q4_DEVINL uint2 codes_int8(uint32_t w) {
     return make_uint2(pack_bf16x2(c[0], c[1]), pack_bf16x2(c[2], c[3]));
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(kThreads, 1)
+// PC: one scale group per tile (per-output-channel scales): the scale is applied once when
+// the tile ends, so the epilogue keeps no accumulators and four epilogue warps suffice;
+// the freed warps dequantize (int8 -> bf16 is the costlier conversion).
+template <int BITS, bool PC>
+__global__ void __launch_bounds__(PC ? kThreadsPC : kThreads, 1)
 prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmp) {
     constexpr int PB = kBM * kBK * BITS / 8;  // payload bytes per k-step (4 or 8 KB)
     constexpr int PROW = kBK * BITS / 8;      // payload bytes per row per k-step (32 or 64)
+    constexpr int NDQW = PC ? 4 : 2;          // dequantizing warps (warps 2 .. 1 + NDQW)
+    constexpr int RPT = 4 / NDQW;             // weight rows per dequantizing thread
+    constexpr int NEPW = PC ? 4 : 8;          // epilogue warps (the rest)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *xs = smem;                                   // kStages x 32 KB
@@ -168,15 +197,15 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(full + i, 1);
-            mbar_init(empty + i, 1 + kDqThreads / 32);  // MMA commit + dequant warps
+            mbar_init(empty + i, 1 + NDQW);  // MMA commit + dequantizing warps
         }
         for (int i = 0; i < kAStages; ++i) {
-            mbar_init(afull + i, kDqThreads / 32);
+            mbar_init(afull + i, NDQW);
             mbar_init(aempty + i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(dfull + i, 1);
-            mbar_init(dempty + i, kEpiWarps);
+            mbar_init(dempty + i, NEPW);
         }
         mbar_init(done, 1);
         fence_barrier_init();
@@ -191,15 +220,15 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
     const uint32_t tmem = *tmem_slot;
 
     bool timed_out = false;
-    const int ntile_cta = a.tiles > (int)blockIdx.x ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int ntile_cta = a.items > (int)blockIdx.x ? (a.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int it = 0;
             for (int tl = 0; tl < ntile_cta; ++tl) {
-                const int tile = blockIdx.x + tl * gridDim.x;
-                const int n0 = (tile % a.tiles_n) * kBM, m0 = (tile / a.tiles_n) * kBN;
+                const Item itm = item_of(a, blockIdx.x + tl * gridDim.x);
+                const int n0 = itm.n0, m0 = itm.m0;
                 for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
                     const int s = it % kStages;
                     if (it >= kStages && !timed_out)
@@ -217,6 +246,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
         if (lane == 0) {
             int it = 0, ait = 0, grp = 0;
             for (int tl = 0; tl < ntile_cta && !timed_out; ++tl) {
+                const Item itm = item_of(a, blockIdx.x + tl * gridDim.x);
+                const uint32_t idesc = (kIdesc & ~(0x3Fu << 17)) | ((uint32_t)(itm.width >> 3) << 17);
                 for (int ks = 0; ks < a.ksteps; ++ks, ++it, ++ait) {
                     const int s = it % kStages, sa = ait % kAStages;
                     const int kg = ks % a.kpg, d = grp & 1;
@@ -230,7 +261,7 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         umma_bf16(dt, sw128_desc(as + sa * kABytes + kk * 32), sw128_desc(xs + s * kXBytes + kk * 32),
-                                  kIdesc, (kg > 0 || kk > 0) ? 1u : 0u);
+                                  idesc, (kg > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(empty + s);
                     umma_commit(aempty + sa);
@@ -242,9 +273,9 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
             }
             umma_commit(done);
         }
-    } else if (warp < 4) {
+    } else if (warp < 2 + NDQW) {
         // ---------------- dequantize: payload -> bf16 codes (A) ----------------
-        const int dt = threadIdx.x - 64;  // 0..63: rows dt and dt + 64
+        const int dt = threadIdx.x - 64;  // rows dt + 32 * NDQW * h, h < RPT
         int it = 0, ait = 0;
         for (int tl = 0; tl < ntile_cta && !timed_out; ++tl) {
             for (int ks = 0; ks < a.ksteps; ++ks, ++it, ++ait) {
@@ -256,8 +287,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 const uint8_t *pst = ps + s * kPBytesMax;
                 uint8_t *ast = as + sa * kABytes;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = dt + 64 * h;
+                for (int h = 0; h < RPT; ++h) {
+                    const int r = dt + 32 * NDQW * h;
                     const uint4 *src = reinterpret_cast<const uint4 *>(pst + r * PROW);
                     uint8_t *dst = ast + r * 128;
                     if constexpr (BITS == 4) {
@@ -283,6 +314,38 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 }
             }
         }
+    } else if constexpr (PC) {
+        // ---------------- epilogue, one group per tile: y = scale * D ----------------
+        const int q = warp & 3;
+        const int rl = 32 * q + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        for (int tl = 0; tl < ntile_cta && !timed_out; ++tl) {
+            const Item itm = item_of(a, blockIdx.x + tl * gridDim.x);
+            const int n = itm.n0 + rl, d = tl & 1;
+            const float sc = a.scales[min(n, a.N - 1)];
+            timed_out = !mbar_wait(dfull + d, (uint32_t)((tl >> 1) & 1));
+            if (timed_out) break;
+            tc_fence_after();
+            for (int ch = 0; ch < kBN / 32; ++ch) {
+                if (32 * ch >= itm.width) break;
+                uint32_t v0[16], v1[16];
+                tmem_ld16(lane_base + (uint32_t)(d * kBN + 32 * ch), v0);
+                tmem_ld16(lane_base + (uint32_t)(d * kBN + 32 * ch + 16), v1);
+                tmem_wait_ld();
+                if (n < a.N) {
+                    const int mb = itm.m0 + 32 * ch, lim = min(itm.width - 32 * ch, a.M - mb);
+                    float *yp = a.y + (size_t)mb * a.N + n;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (i < lim) yp[(size_t)i * a.N] = sc * __uint_as_float(v0[i]);
+                        if (16 + i < lim) yp[(size_t)(16 + i) * a.N] = sc * __uint_as_float(v1[i]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dempty + d);
+        }
     } else {
         // ---------------- epilogue: promotion and stores ----------------
         const int q = warp & 3, half = (warp - 4) >> 2;
@@ -290,8 +353,9 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half);
         int grp = 0;
         for (int tl = 0; tl < ntile_cta && !timed_out; ++tl) {
-            const int tile = blockIdx.x + tl * gridDim.x;
-            const int n0 = (tile % a.tiles_n) * kBM, m0 = (tile / a.tiles_n) * kBN;
+            const Item itm = item_of(a, blockIdx.x + tl * gridDim.x);
+            const int n0 = itm.n0, m0 = itm.m0;
+            const int ncols = min(max(itm.width - 128 * half, 0), 128);  // this warp's valid columns
             const int n = n0 + rl;
             const float *srow = a.scales + (size_t)min(n, a.N - 1) * a.scales_per_row;
             float acc[128];
@@ -307,12 +371,17 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 if (timed_out) break;
                 tc_fence_after();
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t v[16];
-                    tmem_ld16(lane_base + (uint32_t)(d * kBN + 16 * ch), v);
+                for (int ch = 0; ch < 4; ++ch) {
+                    if (32 * ch >= ncols) break;  // narrow item: no more columns here
+                    uint32_t v0[16], v1[16];      // two loads in flight per wait
+                    tmem_ld16(lane_base + (uint32_t)(d * kBN + 32 * ch), v0);
+                    tmem_ld16(lane_base + (uint32_t)(d * kBN + 32 * ch + 16), v1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[16 * ch + i] = fmaf(sc, __uint_as_float(v[i]), acc[16 * ch + i]);
+                    for (int i = 0; i < 16; ++i) {
+                        acc[32 * ch + i] = fmaf(sc, __uint_as_float(v0[i]), acc[32 * ch + i]);
+                        acc[32 * ch + 16 + i] = fmaf(sc, __uint_as_float(v1[i]), acc[32 * ch + 16 + i]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -323,7 +392,7 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
 #pragma unroll
                 for (int i = 0; i < 128; ++i) {
                     const int m = m0 + 128 * half + i;
-                    if (m < a.M) a.y[(size_t)m * a.N + n] = acc[i];
+                    if (i < ncols && m < a.M) a.y[(size_t)m * a.N + n] = acc[i];
                 }
             }
         }
@@ -406,11 +475,19 @@ cudaError_t launch_prefill(const void *x, int64_t M, const uint8_t *payload, con
     a.tiles_n = (int)((N + kBM - 1) / kBM);
     a.tiles = a.tiles_n * (int)((M + kBN - 1) / kBN);
     const int grid = a.tiles < sms ? a.tiles : sms;
+    // complete rounds of whole tiles; the last partial round is cut in 2 or 4 along the
+    // activation rows when the pieces still fit in one round
+    a.full_items = a.tiles / grid * grid;
+    const int rem = a.tiles - a.full_items;
+    a.split = rem == 0 ? 1 : rem * 4 <= grid ? 4 : rem * 2 <= grid ? 2 : 1;
+    a.items = a.full_items + rem * a.split;
     const size_t smem = smem_bytes();
-    auto kern = bits == 4 ? prefill_gemm<4> : prefill_gemm<8>;
+    const bool pc = a.kpg == a.ksteps;  // one scale group per tile
+    auto kern = bits == 4 ? (pc ? prefill_gemm<4, true> : prefill_gemm<4, false>)
+                          : (pc ? prefill_gemm<8, true> : prefill_gemm<8, false>);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, smem, st>>>(a, tmx, tmp);
+    kern<<<grid, pc ? kThreadsPC : kThreads, smem, st>>>(a, tmx, tmp);
     return cudaGetLastError();
 }
 

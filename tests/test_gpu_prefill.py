@@ -66,6 +66,18 @@ def test_ragged_shapes(q4, bits, group):
         check(q4, w, x, bits, group, what=f"M{M} N{N} int{bits} g{group}")
 
 
+@pytest.mark.parametrize("bits,group", [(4, 128), (8, 256)])
+def test_last_round_split_into_narrow_items(q4, bits, group):
+    # 75 x 2 = 150 output tiles on a 148-SM grid: the 2 tiles of the last round are cut
+    # into 4 narrower items each (64 activation rows); all of y is checked on sampled rows
+    rng = np.random.default_rng(21 + bits)
+    N, K, M = 128 * 75, 256, 512
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    x = bf16(rng.normal(0, 1, (M, K)))
+    rows = sorted(set(range(0, 128)) | set(range(N - 256, N)) | set(rng.choice(N, 200, replace=False).tolist()))
+    check(q4, w, x, bits, group, rows=rows, what=f"split int{bits} g{group}")
+
+
 def test_one_hot_rows_select_dequantized_weights_exactly(q4):
     # x = e_k (exact in bf16): the MMA sum is the single code, times the group scale once,
     # so y[:, n] is w'[n, k] bit for bit -- any mix-up of k inside a tile shows here
