@@ -19,10 +19,13 @@
 //               into a 4-deep ring (full/empty mbarriers);
 //   warp 1      allocates tensor memory; one lane issues the MMAs (4 per k-step) and the
 //               tcgen05.commit arrivals that free ring slots and publish finished groups;
-//   warps 2-3   dequantize the payload tile (64 rows each, 2 per thread) into a 3-deep ring
-//               of A tiles, made visible to the tensor core with fence.proxy.async;
+//   warps 2-3   dequantize the payload tile (two rows per thread) into a 3-deep ring of A
+//               tiles, made visible to the tensor core with fence.proxy.async;
 //   warps 4-11  epilogue: warp w reads tensor-memory lanes 32*(w%4).. and 128 of the 256
 //               columns, keeps them as fp32 accumulators, stores y at the end of a tile.
+// With one scale per output channel (one group per tile) the scale is applied once at the
+// end, the epilogue needs no accumulators and 4 warps (10-13), and warps 2-9 dequantize
+// (consecutive threads take consecutive 16-byte chunks of the payload tile).
 // Every wait is bounded (about one second); one that gives up sets Q4_STATUS_TIMEOUT in the
 // status word, and the roles run to completion without further waits.
 #include <cuda.h>
@@ -40,7 +43,7 @@ constexpr int kBK = 64;           // k per step: one 128-byte swizzle row of bf1
 constexpr int kStages = 4;        // x + payload ring
 constexpr int kAStages = 3;       // dequantized A ring
 constexpr int kThreads = 384;     // grouped scales: TMA, MMA, 2 dequantizing, 8 epilogue warps
-constexpr int kThreadsPC = 320;   // one scale per output channel: TMA, MMA, 4 + 4
+constexpr int kThreadsPC = 448;   // one scale per output channel: TMA, MMA, 8 dequantizing, 4 epilogue
 constexpr int kXBytes = kBN * kBK * 2;        // 32 KB
 constexpr int kABytes = kBM * kBK * 2;        // 16 KB
 constexpr int kPBytesMax = kBM * kBK;         // 8 KB (int8); int4 uses half
@@ -176,8 +179,9 @@ __global__ void __launch_bounds__(PC ? kThreadsPC : kThreads, 1)
 prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmp) {
     constexpr int PB = kBM * kBK * BITS / 8;  // payload bytes per k-step (4 or 8 KB)
     constexpr int PROW = kBK * BITS / 8;      // payload bytes per row per k-step (32 or 64)
-    constexpr int NDQW = PC ? 4 : 2;          // dequantizing warps (warps 2 .. 1 + NDQW)
-    constexpr int RPT = 4 / NDQW;             // weight rows per dequantizing thread
+    constexpr int NDQW = PC ? 8 : 2;          // dequantizing warps (warps 2 .. 1 + NDQW)
+    constexpr int NCH = PROW / 16;            // 16-byte payload chunks per row and k-step
+    constexpr int UPT = kBM * NCH / (32 * NDQW);  // payload chunks per dequantizing thread
     constexpr int NEPW = PC ? 4 : 8;          // epilogue warps (the rest)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -275,7 +279,7 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
         }
     } else if (warp < 2 + NDQW) {
         // ---------------- dequantize: payload -> bf16 codes (A) ----------------
-        const int dt = threadIdx.x - 64;  // rows dt + 32 * NDQW * h, h < RPT
+        const int dt = threadIdx.x - 64;  // payload chunks dt + 32 * NDQW * i, i < UPT
         int it = 0, ait = 0;
         for (int tl = 0; tl < ntile_cta && !timed_out; ++tl) {
             for (int ks = 0; ks < a.ksteps; ++ks, ++it, ++ait) {
@@ -286,23 +290,51 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 if (timed_out) break;
                 const uint8_t *pst = ps + s * kPBytesMax;
                 uint8_t *ast = as + sa * kABytes;
+                if constexpr (PC) {
+                    // consecutive threads take consecutive 16-byte payload chunks (conflict-free
+                    // reads); chunk c of row r becomes 4 (int4) or 2 (int8) 16-byte chunks of
+                    // the swizzled A row, which 8 neighbouring threads spread over all banks
+    #pragma unroll
+                    for (int i = 0; i < UPT; ++i) {
+                        const int u = dt + 32 * NDQW * i;
+                        const int r = u / NCH, c = u % NCH;
+                        const uint4 p = *reinterpret_cast<const uint4 *>(pst + r * PROW + 16 * c);
+                        const uint32_t wd[4] = {p.x, p.y, p.z, p.w};
+                        uint8_t *dst = ast + r * 128;
+                        if constexpr (BITS == 4) {
+    #pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<uint4 *>(dst + (((4 * c + q) ^ (r & 7)) << 4)) = codes_int4(wd[q]);
+                        } else {
+    #pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const uint2 lo = codes_int8(wd[2 * q]), hi = codes_int8(wd[2 * q + 1]);
+                                *reinterpret_cast<uint4 *>(dst + (((2 * c + q) ^ (r & 7)) << 4)) =
+                                    make_uint4(lo.x, lo.y, hi.x, hi.y);
+                            }
+                        }
+                    }
+                } else {
+                    // two whole rows per thread (rows dt and dt + 64)
 #pragma unroll
-                for (int h = 0; h < RPT; ++h) {
-                    const int r = dt + 32 * NDQW * h;
-                    const uint4 *src = reinterpret_cast<const uint4 *>(pst + r * PROW);
-                    uint8_t *dst = ast + r * 128;
-                    if constexpr (BITS == 4) {
-                        const uint4 p0 = src[0], p1 = src[1];  // 64 codes
-                        const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = dt + 64 * h;
+                        const uint4 *src = reinterpret_cast<const uint4 *>(pst + r * PROW);
+                        uint8_t *dst = ast + r * 128;
+                        if constexpr (BITS == 4) {
+                            const uint4 p0 = src[0], p1 = src[1];  // 64 codes
+                            const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = codes_int4(wds[c]);
-                    } else {
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = codes_int4(wds[c]);
+                        } else {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint2 wv = reinterpret_cast<const uint2 *>(src)[c];  // 8 codes
-                            const uint2 lo = codes_int8(wv.x), hi = codes_int8(wv.y);
-                            *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                            for (int c = 0; c < 8; ++c) {
+                                const uint2 wv = reinterpret_cast<const uint2 *>(src)[c];  // 8 codes
+                                const uint2 lo = codes_int8(wv.x), hi = codes_int8(wv.y);
+                                *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) =
+                                    make_uint4(lo.x, lo.y, hi.x, hi.y);
+                            }
                         }
                     }
                 }
