@@ -118,6 +118,12 @@ Q4_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr)
         : "memory");
 }
+// acc (a pair of fp32 in one 64-bit register) += s2 * (lo, hi), one packed instruction.
+Q4_DEVINL void fma2_acc(uint64_t &acc, uint64_t s2, uint32_t lo, uint32_t hi) {
+    asm("{\n\t.reg .b64 v;\n\tmov.b64 v, {%1, %2};\n\tfma.rn.f32x2 %0, %3, v, %0;\n\t}"
+        : "+l"(acc)
+        : "r"(lo), "r"(hi), "l"(s2));
+}
 Q4_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
 Q4_DEVINL void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -390,14 +396,15 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
             const int ncols = min(max(itm.width - 128 * half, 0), 128);  // this warp's valid columns
             const int n = n0 + rl;
             const float *srow = a.scales + (size_t)min(n, a.N - 1) * a.scales_per_row;
-            float acc[128];
+            uint64_t acc[64];  // 128 fp32 accumulators, two per register pair
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+            for (int i = 0; i < 64; ++i) acc[i] = 0ull;
             const int ngroups = a.ksteps / a.kpg;
             float s_next = srow[0];
             for (int gi = 0; gi < ngroups; ++gi, ++grp) {
                 const int d = grp & 1;
                 const float sc = s_next;
+                const uint64_t s2 = ((uint64_t)__float_as_uint(sc) << 32) | __float_as_uint(sc);
                 if (gi + 1 < ngroups) s_next = srow[gi + 1];
                 if (!timed_out) timed_out = !mbar_wait(dfull + d, (uint32_t)((grp >> 1) & 1));
                 if (timed_out) break;
@@ -410,9 +417,9 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                     tmem_ld16(lane_base + (uint32_t)(d * kBN + 32 * ch + 16), v1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        acc[32 * ch + i] = fmaf(sc, __uint_as_float(v0[i]), acc[32 * ch + i]);
-                        acc[32 * ch + 16 + i] = fmaf(sc, __uint_as_float(v1[i]), acc[32 * ch + 16 + i]);
+                    for (int i = 0; i < 8; ++i) {
+                        fma2_acc(acc[16 * ch + i], s2, v0[2 * i], v0[2 * i + 1]);
+                        fma2_acc(acc[16 * ch + 8 + i], s2, v1[2 * i], v1[2 * i + 1]);
                     }
                 }
                 tc_fence_before();
@@ -424,7 +431,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
 #pragma unroll
                 for (int i = 0; i < 128; ++i) {
                     const int m = m0 + 128 * half + i;
-                    if (i < ncols && m < a.M) a.y[(size_t)m * a.N + n] = acc[i];
+                    const uint32_t bits = (i & 1) ? (uint32_t)(acc[i >> 1] >> 32) : (uint32_t)acc[i >> 1];
+                    if (i < ncols && m < a.M) a.y[(size_t)m * a.N + n] = __uint_as_float(bits);
                 }
             }
         }
