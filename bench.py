@@ -18,6 +18,8 @@ roofline = the kernel with the largest share of step time, timed with CUDA event
 e2e      = the same step through the public API from pinned host buffers, with the H2D
            copy of W and x and the D2H copy of every y inside the timed region.
 prefill  = the M = 2048 bf16 prefill qgemm (K = 4096, N = 14336) in TFLOP/s.
+decode_stack = the 224 GEMVs of a Llama-7B-shaped stack per token step, one CUDA graph per
+           step, at M = 1, 4, 16 (int4 g128 and int8 per channel): us per step and GB/s.
 cpu_baseline = the oracle (single-threaded C) on a bounded sample of the same step.
 
 --impl reference times the oracle alone on that sample (there is no reference
@@ -422,6 +424,8 @@ def run_ours(args):
         out["e2e"] = e2e(args, q4, dev, w_host, x_host, N, K, formats, Ms, bytes_per_step, world)
     if rank == 0 and not args.no_prefill:
         out["prefill"] = prefill(args, q4, dev, peaks, peak_kind)
+    if rank == 0 and not args.no_stack:
+        out["decode_stack"] = decode_stack_section(args, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, el, desc = oracle_sample(N, K, formats, Ms, budget_s=args.cpu_seconds)
         out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": host_cores_used(),
@@ -510,6 +514,20 @@ def prefill(args, q4, dev, peaks, peak_kind):
             "peak_bf16_tflops": peaks["bf16_tflops"], **res}
 
 
+def decode_stack_section(args, dev):
+    """The 224-GEMV Llama-7B-shaped stack, one CUDA graph per token step (M = 1, 4, 16)."""
+    from int4_quantized_b200 import decode_stack as ds
+
+    out = {"workload": "Llama-7B-shaped linear stack: 32 x (4 x 4096x4096, 2 x 11008x4096, 4096x11008), "
+                       "W ~ N(0, 0.02) drawn on the device, weights read from HBM every step",
+           "gemvs_per_step": 7 * 32}
+    for bits, group, key in ((4, 128, "int4_g128"), (8, None, "int8_per_channel")):
+        stack = ds.build_stack(bits, group, 32, dev)
+        out[key] = [ds.time_stack(stack, bits, M, reps=10) for M in (1, 4, 16)]
+        del stack
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,6 +538,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stack", action="store_true", help="skip the whole-stack decode section")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
