@@ -249,10 +249,14 @@ def config_block():
 
 
 # ----------------------------------------------------------------------------------------
-def kernel_source_sha():
+# the sources each bench kernel is built from (the traffic figures are dropped when any changes)
+KERNEL_SOURCES = {"qpack": ("qpack.cu", "common.cuh", "kernels.h"), "gemv": ("gemv.cu", "common.cuh", "kernels.h")}
+
+
+def kernel_source_sha(kernel_key):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int4_quantized_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    for fn in KERNEL_SOURCES[kernel_key.split("_")[0]]:
         with open(os.path.join(d, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -260,16 +264,16 @@ def kernel_source_sha():
 
 def ncu_traffic(kernel_key):
     """DRAM bytes per launch for `kernel_key` from the committed ncu summary, or None when
-    the summary is missing or the kernel sources changed since it was taken."""
+    the summary is missing or the kernel's sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_sha") != kernel_source_sha():
-        return None
     v = d.get("kernels", {}).get(kernel_key)
-    return None if v is None else v.get("dram_bytes_per_launch")
+    if v is None or v.get("source_sha") != kernel_source_sha(kernel_key):
+        return None
+    return v.get("dram_bytes_per_launch")
 
 
 def run_ours(args):
