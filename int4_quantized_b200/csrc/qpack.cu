@@ -176,10 +176,43 @@ __global__ void __launch_bounds__(256, 2) qpack_chunk(const float *__restrict__ 
 #pragma unroll
             for (int off = 1; off < LPG; off <<= 1) m[u] = fmaxf(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
         }
+        // The scale and reciprocal of each group are computed once, by one lane per
+        // group (lane L takes group L, L + 32, ...), and handed back by shuffles; the
+        // division and reciprocal are the same IEEE operations whichever lane does them.
+        constexpr int NGC = CH / G;                 // groups in the chunk
+        constexpr int GPL = G >= 128 ? 1 : 128 / G; // groups per load (when G < 128)
+        constexpr int NR = (NGC + 31) / 32;         // groups per lane
+        float s_own[NR], r_own[NR];
+        bool fast_own[NR];
+#pragma unroll
+        for (int rr = 0; rr < NR; ++rr) {
+            const int gi = lane + 32 * rr;          // the group this lane computes
+            const int ug = G >= 128 ? gi * UPG : gi / GPL;  // its first load
+            const int lp = G >= 128 ? 0 : (gi % GPL) * LPG; // a lane holding its max
+            float mg = 0.f;
+#pragma unroll
+            for (int u = 0; u < U; u += UPG) {
+                const float t = __shfl_sync(0xffffffffu, m[u], lp);
+                mg = (u == ug) ? t : mg;
+            }
+            const float sc = scale_of_f<BITS>(mg);
+            const GroupDiv dd = make_div(sc);
+            s_own[rr] = sc;
+            r_own[rr] = dd.r;
+            fast_own[rr] = dd.fast;
+            if (gi < NGC) scales[c * NGC + gi] = sc;
+        }
 #pragma unroll
         for (int u = 0; u < U; u += UPG) {
-            const float s = scale_of_f<BITS>(m[u]);
-            const GroupDiv d = make_div(s);
+            // this lane's group in load u, and the lane that computed it
+            // (the groups of one load never straddle a multiple of 32, so the register
+            // set rr is the same in every lane and in the source lane)
+            const int gi = G >= 128 ? u / UPG : u * GPL + lane / LPG;
+            const int rr = (G >= 128 ? u / UPG : u * GPL) / 32, src = gi % 32;
+            GroupDiv d;
+            d.s = __shfl_sync(0xffffffffu, s_own[NR > 1 ? rr : 0], src);
+            d.r = __shfl_sync(0xffffffffu, r_own[NR > 1 ? rr : 0], src);
+            d.fast = __shfl_sync(0xffffffffu, (int)fast_own[NR > 1 ? rr : 0], src) != 0;
 #pragma unroll
             for (int q = 0; q < UPG; ++q) {
                 const int uu = u + q;
@@ -191,8 +224,6 @@ __global__ void __launch_bounds__(256, 2) qpack_chunk(const float *__restrict__ 
                 else
                     reinterpret_cast<uint32_t *>(my)[e] = pack4<8>(t);
             }
-            // one scale per group: the groups of this load (or load range), in order
-            if (lane % LPG == 0) scales[(c * CH + 128 * u + 4 * lane) / G] = s;
         }
         __syncwarp();
         uint8_t *dst = payload + c * CB;
