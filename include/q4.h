@@ -147,8 +147,9 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
  * finite inputs (y_exact = the fp64 sum).
  * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0, group divides K and
- * group % 32 == 0 (per-channel scales are group = K). M, N >= 0; M == 0 or
- * N == 0 enqueues nothing.
+ * group % 32 == 0 (per-channel scales are group = K); N, K <= 2^30 and, on
+ * the fused GEMV path, M <= 1048560 (65535 chunks of 16 rows). M, N >= 0;
+ * M == 0 or N == 0 enqueues nothing.
  * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
  * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
  */

@@ -441,6 +441,22 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         // ---------------- producer warp ----------------
         const uint8_t *fsrc = a.frag + (size_t)mc * a.stages_total * a.fslot_bytes;
         const int primed = min(nst, nring);
+        // The first `primed` stages' digits are copied once gemv_prep has finished, so that
+        // the codes of those stages stream in meanwhile; `issued` of them have gone out.
+        // They go out before any wait on the consumers, who need them to make progress.
+        int issued = 0;
+        auto issue_primed = [&](int upto) {
+            if (issued >= upto) return;
+            if (issued == 0) grid_dep_wait();
+            if (lane == 0 && !timed_out) {
+                const uint32_t fb = (uint32_t)a.fslot_bytes;
+                for (int q = issued; q < upto; ++q) {
+                    mbar_arrive_expect_tx(ffull + q, fb);
+                    bulk_copy_g2s(fslots + q * fb, fsrc + (size_t)(st_lo + q) * fb, fb, ffull + q);
+                }
+            }
+            issued = upto;
+        };
         int slot = 0, round = 0;          // ring position, completed passes over the ring
         int eb = eb_first, eb_left = 0;   // current k-block, stages left in it
         for (int ks = 0; ks < nst; ++ks) {
@@ -450,7 +466,12 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                 if (ks > 0) ++eb;
                 eb_left = min(a.ebs * (eb + 1), st_hi) - s;
                 const int ebl = eb - eb_first, b = ebl & 1;
-                if (ebl >= 2 && !timed_out) timed_out = !mbar_wait(sempty + b, (uint32_t)(((ebl >> 1) - 1) & 1));
+                if (ebl >= 2) {
+                    // the consumers release this buffer only after the digits of the
+                    // stages before this one have reached them
+                    if constexpr (!INK) issue_primed(min(ks, primed));
+                    if (!timed_out) timed_out = !mbar_wait(sempty + b, (uint32_t)(((ebl >> 1) - 1) & 1));
+                }
                 int gA, ng;
                 eb_groups(eb, gA, ng);
                 // asynchronous copies: the producer never waits for them; rows past N copy
@@ -489,16 +510,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                         bulk_copy_g2s(fslots + slot * fb, fsrc + (size_t)s * fb, fb, ffull + slot);
                     }
                 }
-                if (ks == primed - 1) {
-                    // the ring is primed with codes; the digits come from gemv_prep
-                    grid_dep_wait();
-                    if (lane == 0 && !timed_out) {
-                        for (int q = 0; q < primed; ++q) {
-                            mbar_arrive_expect_tx(ffull + q, fb);
-                            bulk_copy_g2s(fslots + q * fb, fsrc + (size_t)(st_lo + q) * fb, fb, ffull + q);
-                        }
-                    }
-                }
+                if (ks == primed - 1) issue_primed(primed);  // the ring is primed with codes
             }
             if (++slot == nring) { slot = 0; ++round; }
         }
@@ -866,7 +878,7 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
         if (p.gps == 1) p.gps = 0;  // one group per stage: the same as a stage inside a group
         if (p.gps < 0) p.L = bits == 4 ? 4 : 8;
     }
-    if (K > ((int64_t)1 << 30) || N > ((int64_t)1 << 30) || M > ((int64_t)1 << 20)) return false;
+    if (K > ((int64_t)1 << 30) || N > ((int64_t)1 << 30) || M > (int64_t)65535 * 16) return false;
     p.segk = 32 * p.L / bits;
     p.segs = (int)(K / p.segk);
     p.spg = (int)(group / p.segk);

@@ -29,8 +29,11 @@ def run_bf16(q4, x_bf16, payload, scales, N, K, bits, group):
     import torch
 
     xt = x_bf16.cuda()
-    y = q4.qgemm(xt, torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda(), N, K, bits, group)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.qgemm(xt, torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda(), N, K, bits, group,
+                 status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"status word {int(status.item()):#x}: a bounded wait gave up"
     return y.cpu().numpy()
 
 

@@ -31,8 +31,11 @@ def run_gpu(q4, x, payload, scales, N, K, bits, group, bf16=False):
     xt = torch.from_numpy(x).cuda()
     if bf16:
         xt = xt.to(torch.bfloat16)
-    y = q4.qgemm(xt, torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda(), N, K, bits, group)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.qgemm(xt, torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda(), N, K, bits, group,
+                 status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"status word {int(status.item()):#x}: a bounded wait gave up"
     return y.cpu().numpy()
 
 
@@ -126,6 +129,32 @@ def test_group_variants(q4, bits, group, M):
     w.reshape(-1)[rng.choice(N * K, 50, replace=False)] *= 20  # outliers
     x = rng.normal(0, 1, (M, K)).astype(np.float32)
     case(q4, w, x, bits, group, what=f"int{bits} g{group} M{M}")
+
+
+@pytest.mark.parametrize("bits,group,K", [(4, 64, 4160), (4, 32, 4128), (8, 32, 4128), (8, 96, 4128 + 96 * 3)])
+@pytest.mark.parametrize("M", [1, 3, 9])
+def test_partial_last_stage(q4, bits, group, K, M):
+    # rows whose byte length is not a multiple of the 128-byte stage: the last stage of
+    # every row is partly outside the payload
+    if K % group:
+        K = group * (K // group)
+    rng = np.random.default_rng(K + bits + M)
+    w = rng.normal(0, 0.02, (136, K)).astype(np.float32)
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    case(q4, w, x, bits, group, what=f"K{K} int{bits} g{group} M{M}")
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (8, 32), (4, 64), (4, 128)])
+@pytest.mark.parametrize("M", [2, 9])
+def test_many_k_blocks_per_cta(q4, bits, group, M):
+    # 152 x 128 output rows fill the grid without a K split: each CTA streams all of K
+    # through its rings, crossing many k-blocks (scale buffers reused several times)
+    # before and after its ring of codes and digits wraps
+    N, K = 152 * 128, 2048
+    rng = np.random.default_rng(bits * 100 + group + M)
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    case(q4, w, x, bits, group, rows=sample_rows(N, 200, M), what=f"int{bits} g{group} M{M}")
 
 
 @pytest.mark.parametrize("M", [1, 16, 40, 64, 128])
