@@ -245,6 +245,8 @@ def config_block():
     return {"workload": "4096x4096 W~N(0,0.02)+0.1% 20x outliers; qpack int4 g128 + int8 g128; GEMV M=1 and M=8",
             "N": 4096, "K": 4096, "formats": ["int4 g128", "int8 g128"], "M": list(wl.Ms),
             "l2": f"inputs rotate over {ROT} copies (>126 MB L2); each GEMV reads payload written 2 steps earlier",
+            "gemv_weights": "static during the step (packed 2 steps earlier): GEMVs are launched with "
+                            "Q4_QGEMM_WEIGHTS_STATIC and stream them while the previous kernel ends",
             "parallelism": "replicas (one independent problem per GPU)"}
 
 
@@ -316,7 +318,9 @@ def run_ours(args):
         if kind == "qpack":
             q4.qpack(W[wi], f[0], f[1], payload=P[f][wi], scales=S[f][wi])
         else:
-            q4.qgemm(X[M], P[f][gj], S[f][gj], N, K, f[0], f[1], out=Y[(f, M)], workspace=WS[(f, M)])
+            # the payload read here was packed two steps earlier: static while this step runs
+            q4.qgemm(X[M], P[f][gj], S[f][gj], N, K, f[0], f[1], out=Y[(f, M)], workspace=WS[(f, M)],
+                     weights_static=True)
 
     plan = []
     for f in formats:
@@ -428,6 +432,8 @@ def run_ours(args):
         out["e2e"] = e2e(args, q4, dev, w_host, x_host, N, K, formats, Ms, bytes_per_step, world)
     if rank == 0 and not args.no_prefill:
         out["prefill"] = prefill(args, q4, dev, peaks, peak_kind)
+    if rank == 0 and not args.no_mlp70b:
+        out["mlp70b"] = mlp70b_section(args, dev, peaks)
     if rank == 0 and not args.no_stack:
         out["decode_stack"] = decode_stack_section(args, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -518,6 +524,78 @@ def prefill(args, q4, dev, peaks, peak_kind):
             "peak_bf16_tflops": peaks["bf16_tflops"], **res}
 
 
+def mlp70b_section(args, dev, peaks):
+    """The 70B-shaped MLP matrices (gate/up 28672x8192, down 8192x28672, int4 g64, M = 1).
+
+    Each matrix is packed once on the GPU. Two CUDA graphs of back-to-back calls: rounds of
+    (gate, up), which share a shape, and rounds of (gate, up, down); every call reads
+    another 132 MB matrix than the call before it, and a round (264 or 396 MB) is past the
+    126 MB L2, so the weights come from HBM. The first graph gives the 28672x8192 time per
+    call, the second the time of the three; the 8192x28672 time is their difference
+    (marked "derived"). Both launch modes are timed: plain stream order, and weights
+    declared static.
+    """
+    import torch
+
+    import int4_quantized_b200 as q4
+
+    wl = workloads.WORKLOADS["mlp70b"]
+    bits, group = wl.formats[0]
+    mats = []
+    for m in wl.matrices:
+        w = torch.from_numpy(workloads.weight(m)).to(dev)
+        payload, scales = q4.qpack(w, bits, group)
+        del w
+        x = torch.from_numpy(workloads.activations(1, m.K, wl.x_seed(m.K))).to(dev)
+        y = torch.empty((1, m.N), dtype=torch.float32, device=dev)
+        mats.append((m, payload, scales, x, y, payload.numel() + 4 * scales.numel()))
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    nb = mats[0][5]
+    rounds = 10
+
+    def graph_time(seq, static):
+        def run():
+            for _ in range(rounds):
+                for m, p, sc, x, y, _ in seq:
+                    q4.qgemm(x, p, sc, m.N, m.K, bits, group, out=y, weights_static=static)
+        with torch.cuda.stream(stream):
+            run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        ts = []
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+            for _ in range(5):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                b.synchronize()
+                ts.append(a.elapsed_time(b) * 1e3 / rounds)
+        del g
+        return sorted(ts)[len(ts) // 2]
+
+    def entry(us, nbytes, **kw):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {**kw, "us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+
+    out = {"workload": wl.description, "bytes_per_matrix": nb, "calls_per_graph": {"gate_up": 2 * rounds,
+                                                                                  "all3": 3 * rounds}}
+    for static in (False, True):
+        t_gu = graph_time(mats[:2], static) / 2
+        t_all = graph_time(mats, static)
+        out["int4_g64_static" if static else "int4_g64"] = {
+            "gate_up_28672x8192": entry(t_gu, nb, N=28672, K=8192),
+            "down_8192x28672": entry(t_all - 2 * t_gu, nb, N=8192, K=28672, derived=True),
+            "all3": entry(t_all, 3 * nb),
+        }
+    return out
+
+
 def decode_stack_section(args, dev):
     """The 224-GEMV Llama-7B-shaped stack, one CUDA graph per token step (M = 1, 4, 16)."""
     from int4_quantized_b200 import decode_stack as ds
@@ -527,7 +605,8 @@ def decode_stack_section(args, dev):
            "gemvs_per_step": 7 * 32}
     for bits, group, key in ((4, 128, "int4_g128"), (8, None, "int8_per_channel")):
         stack = ds.build_stack(bits, group, 32, dev)
-        out[key] = [ds.time_stack(stack, bits, M, reps=10) for M in (1, 4, 16)]
+        out[key] = [ds.time_stack(stack, bits, M, reps=10, weights_static=True) for M in (1, 4, 16)]
+        out[key + "_plain"] = [ds.time_stack(stack, bits, M, reps=10, weights_static=False) for M in (1, 4, 16)]
         del stack
     return out
 
@@ -543,6 +622,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-stack", action="store_true", help="skip the whole-stack decode section")
+    ap.add_argument("--no-mlp70b", action="store_true", help="skip the 70B-shaped MLP section")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -147,15 +147,41 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
  * finite inputs (y_exact = the fp64 sum).
  * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0, group divides K and
- * group % 32 == 0 (per-channel scales are group = K); N, K <= 2^30 and, on
- * the fused GEMV path, M <= 1048560 (65535 chunks of 16 rows). M, N >= 0;
- * M == 0 or N == 0 enqueues nothing.
+ * group % 32 == 0 (per-channel scales are group = K); N, K <= 2^30 and
+ * M <= 1048560 (65535 chunks of 16 rows). M, N >= 0; M == 0 or N == 0
+ * enqueues nothing.
  * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
  * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
  */
 Q4_API q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
                 const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
                 void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream);
+
+/* qgemm_ex flags. */
+#define Q4_QGEMM_WEIGHTS_STATIC 1u
+
+/*
+ * qgemm_ex -- qgemm with option flags (the pages have no counterpart: this is a
+ * launch-overlap option for sequences of calls, e.g. the linear layers of one
+ * decode step, whose packed weights stay fixed while the sequence runs).
+ *   flags  0, or Q4_QGEMM_WEIGHTS_STATIC: payload and scales may be read while
+ *          the kernel enqueued before this call on the same stream is still
+ *          running (programmatic dependent launch), so that their streaming
+ *          overlaps that kernel's tail. The caller promises that the last write
+ *          to payload and scales finished before that previous kernel started
+ *          (weights packed once and reused qualify; packing them with the call
+ *          just before does not). x, y, the workspace and the status word keep
+ *          full stream order: every read of x and every write waits until the
+ *          previous kernel has finished. Only the fused GEMV path (not the
+ *          bf16 M >= 64 tensor-core GEMM) uses the flag; the result is bit-for-bit
+ *          the same as without it.
+ *   Other arguments, results and errors as qgemm; unknown flag bits are
+ *   Q4_ERR_ARG. qgemm(...) is qgemm_ex(..., flags = 0, ...).
+ */
+Q4_API q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                void *workspace, size_t workspace_bytes, uint32_t flags, uint32_t *status_word,
+                void *stream);
 
 /* Size of the one device scratch buffer that qgemm_noalloc uses (4 MiB). */
 #define Q4_NOALLOC_SCRATCH_BYTES (4u << 20)

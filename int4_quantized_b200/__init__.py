@@ -25,13 +25,14 @@ import torch
 __all__ = [
     "Q4Error", "lib", "lib_path", "payload_bytes", "num_scales", "qgemm_workspace_bytes",
     "qpack", "qdequant", "qgemm", "qgemm_noalloc", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
-    "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_ERR_SCRATCH_LIMIT", "Q4_X_F32", "Q4_X_BF16", "STATUS_NONFINITE", "STATUS_TIMEOUT",
+    "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_ERR_SCRATCH_LIMIT", "Q4_X_F32", "Q4_X_BF16", "Q4_QGEMM_WEIGHTS_STATIC", "STATUS_NONFINITE", "STATUS_TIMEOUT",
 ]
 
 Q4_OK, Q4_ERR_ARG, Q4_ERR_UNSUPPORTED, Q4_ERR_CUDA, Q4_ERR_NONFINITE, Q4_ERR_WORKSPACE, \
     Q4_ERR_SCRATCH_LIMIT = range(7)
 NOALLOC_SCRATCH_BYTES = 4 << 20  # Q4_NOALLOC_SCRATCH_BYTES
 Q4_X_F32, Q4_X_BF16 = 0, 1
+Q4_QGEMM_WEIGHTS_STATIC = 1
 STATUS_NONFINITE = 1
 STATUS_TIMEOUT = 2
 
@@ -73,6 +74,9 @@ def lib() -> ctypes.CDLL:
                 L.q4_qgemm_workspace_bytes.restype = sz
                 L.qgemm.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, sz, vp, vp]
                 L.qgemm.restype = i32
+                L.qgemm_ex.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, sz, ctypes.c_uint32, vp,
+                                       vp]
+                L.qgemm_ex.restype = i32
                 L.qgemm_noalloc.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, vp]
                 L.qgemm_noalloc.restype = i32
                 _lib = L
@@ -168,8 +172,13 @@ def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
 
 def qgemm(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, N: int, K: int, bits: int,
           group: int, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-          status: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y[M, N] = x[M, K] @ W'^T from the packed codes (x float32 or bfloat16)."""
+          status: Optional[torch.Tensor] = None, weights_static: bool = False) -> torch.Tensor:
+    """y[M, N] = x[M, K] @ W'^T from the packed codes (x float32 or bfloat16).
+
+    weights_static=True (Q4_QGEMM_WEIGHTS_STATIC): payload and scales may be streamed
+    while the previous kernel on the stream still runs; only valid when their last write
+    finished before that kernel started (weights packed once, then reused).
+    """
     _cuda(x, "x")
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("x must be float32 or bfloat16")
@@ -189,8 +198,9 @@ def qgemm(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, N: int, 
     if status is not None:
         _cuda(status, "status", torch.int32)
     with torch.cuda.device(x.device):
-        _check(lib().qgemm(_ptr(x2), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group, _ptr(out),
-                           _ptr(workspace), ws_bytes, _ptr(status), _stream(x.device)), "qgemm")
+        _check(lib().qgemm_ex(_ptr(x2), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group, _ptr(out),
+                              _ptr(workspace), ws_bytes, Q4_QGEMM_WEIGHTS_STATIC if weights_static else 0,
+                              _ptr(status), _stream(x.device)), "qgemm")
     return out
 
 

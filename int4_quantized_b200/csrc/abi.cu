@@ -137,9 +137,11 @@ size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64
     return pl.bytes;
 }
 
-q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
-                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
-                void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream) {
+q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                   const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                   void *workspace, size_t workspace_bytes, uint32_t flags, uint32_t *status_word,
+                   void *stream) {
+    if (flags & ~(uint32_t)Q4_QGEMM_WEIGHTS_STATIC) return Q4_ERR_ARG;
     q4::GemvPlan pl;
     q4_status st = plan_qgemm(M, N, K, bits, group, xt, &pl);
     if (st != Q4_OK) return st;
@@ -154,8 +156,16 @@ q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
     if ((uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
     if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return Q4_ERR_WORKSPACE;
     cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,
-                                    workspace, status_word, as_stream(stream));
+                                    workspace, status_word, (flags & Q4_QGEMM_WEIGHTS_STATIC) != 0,
+                                    as_stream(stream));
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
+                const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
+                void *workspace, size_t workspace_bytes, uint32_t *status_word, void *stream) {
+    return qgemm_ex(x, xt, M, payload, scales, N, K, bits, group, y, workspace, workspace_bytes, 0u,
+                    status_word, stream);
 }
 
 q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,

@@ -212,6 +212,7 @@ Q4_DEVINL uint32_t absmax8(const float (&v)[8]) {
 template <int BITS, int L, bool XBF16>
 __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
     grid_dep_launch();
+    grid_dep_wait();  // x may be the output of the kernel before this one
     constexpr int STAGEK = kTileBytes * 8 / BITS;
     __shared__ int e_sh[16];
     const int eb = blockIdx.x, mc = blockIdx.y;
@@ -400,6 +401,9 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     uint64_t *sempty = sfull + 2;
     float *red = reinterpret_cast<float *>(slots);  // [128][16] partial sums, after the main loop
 
+    // the next call on the stream may start its own prologue (and, when its weights are
+    // declared static, stream them) while this grid runs; it waits before reading x
+    grid_dep_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int crank = (int)(blockIdx.x % (unsigned)a.CS);
     const int cl = (int)(blockIdx.x / (unsigned)a.CS);
@@ -520,7 +524,9 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         const int ct = threadIdx.x;  // 0..255
         if constexpr (INK) {
             // digits of this CTA's K range of the single activation row, built while the
-            // first payload tiles are in flight
+            // first payload tiles are in flight; x may be the output of the kernel before
+            // this one (a no-op unless this grid was launched as a dependent)
+            grid_dep_wait();
             const int nlb = nst > 0 ? (st_hi - 1) / a.ebs - eb_first + 1 : 0;
             for (int i = ct; i < nlb; i += kConsumerThreads) mx_sh[i] = 0;
             named_barrier_sync(1, kConsumerThreads);
@@ -795,16 +801,25 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// early: the weights are static, so the call's first grid may start (and the stream
+// kernel read payload and scales) while the previous kernel on the stream still runs.
+// Every read of x, and every write, still waits for that kernel to finish.
 template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16>
 cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
-                         cudaStream_t st) {
+                         bool early, cudaStream_t st) {
     cudaError_t err;
+    cudaLaunchAttribute pdl;
+    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl.val.programmaticStreamSerializationAllowed = 1;
     if constexpr (!INK) {
-        if (x_bf16)
-            gemv_prep<BITS, L, true><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
-        else
-            gemv_prep<BITS, L, false><<<dim3(pl.n_eb, pl.nmc), 256, 0, st>>>(a);
-        err = cudaGetLastError();
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3(pl.n_eb, pl.nmc);
+        pc.blockDim = dim3(256);
+        pc.stream = st;
+        pc.attrs = &pdl;
+        pc.numAttrs = early ? 1 : 0;
+        err = x_bf16 ? cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, true>, a)
+                     : cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, false>, a);
         if (err != cudaSuccess) return err;
     }
     auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16>;
@@ -821,28 +836,30 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
     attr[0].val.clusterDim.x = pl.CS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    attr[1] = pdl;
     cfg.attrs = attr;
-    cfg.numAttrs = INK ? 1 : 2;  // the in-kernel path reads x at once: no early start
+    // after gemv_prep the stream kernel always starts early (the prep grid itself began
+    // only once everything before it had finished, unless the weights are static); the
+    // one-kernel path starts early only with static weights
+    cfg.numAttrs = INK && !early ? 1 : 2;
     return cudaLaunchKernelEx(&cfg, kern, a, tm);
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
-                          cudaStream_t st) {
+                          bool early, cudaStream_t st) {
 #define Q4_INK(B, LL, G)                                                                         \
     if (pl.bits == B && pl.L == LL && pl.gps == G)                                               \
-        return x_bf16 ? launch_typed<B, LL, 1, G, true, true>(pl, a, tm, true, st)               \
-                      : launch_typed<B, LL, 1, G, true, false>(pl, a, tm, false, st);
+        return x_bf16 ? launch_typed<B, LL, 1, G, true, true>(pl, a, tm, true, early, st)        \
+                      : launch_typed<B, LL, 1, G, true, false>(pl, a, tm, false, early, st);
 #define Q4_STAGED(B, LL, G)                                                                      \
     if (pl.bits == B && pl.L == LL && pl.gps == G) {                                             \
         switch (pl.NB) {                                                                         \
-            case 1: return launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, st);       \
-            case 2: return launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, st);       \
-            case 4: return launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, st);       \
-            default: return launch_typed<B, LL, 8, G, false, false>(pl, a, tm, x_bf16, st);      \
+            case 1: return launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, early, st); \
+            case 2: return launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, early, st); \
+            case 4: return launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, early, st); \
+            default: return launch_typed<B, LL, 8, G, false, false>(pl, a, tm, x_bf16, early, st); \
         }                                                                                        \
     }
 #define Q4_ALL(M)                                                                                \
@@ -937,7 +954,8 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
 
 cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t M,
                         const uint8_t *payload, const float *scales, int64_t N, int64_t K,
-                        int64_t group, float *y, void *ws, uint32_t *status, cudaStream_t st) {
+                        int64_t group, float *y, void *ws, uint32_t *status, bool weights_static,
+                        cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     const uint64_t rowbytes = (uint64_t)K * pl.bits / 8;
@@ -974,7 +992,7 @@ cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t 
     a.paired = pl.paired;
     a.nst_ring = pl.nst_ring;
     a.fslot_bytes = pl.fslot_bytes;
-    return dispatch_gemv(pl, a, tm, x_bf16, st);
+    return dispatch_gemv(pl, a, tm, x_bf16, weights_static, st);
 }
 
 }  // namespace q4

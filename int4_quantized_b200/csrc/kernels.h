@@ -44,7 +44,8 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, int sms
 
 cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t M,
                         const uint8_t *payload, const float *scales, int64_t N, int64_t K,
-                        int64_t group, float *y, void *ws, uint32_t *status, cudaStream_t st);
+                        int64_t group, float *y, void *ws, uint32_t *status, bool weights_static,
+                        cudaStream_t st);
 
 // ---- prefill GEMM (tcgen05) ----------------------------------------------------------
 // bf16 x with M >= 64, K and group multiples of 64: the tensor-memory GEMM of prefill.cu.

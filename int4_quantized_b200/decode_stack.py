@@ -9,6 +9,11 @@ qgemm calls in layer order, captured once in a CUDA graph (launch overhead is wh
 dominates a stack of small GEMVs), and replayed. The stack (3.4 GB packed at int4 g128,
 6.5 GB at int8 per channel) is far larger than L2, so every step reads the weights from
 HBM. Reported: microseconds per token step and the GB/s of packed weights + scales.
+
+With --static (the default) every call declares its weights static
+(Q4_QGEMM_WEIGHTS_STATIC): each GEMV streams its weights while the one before it
+finishes, as they are packed once and never written during the step; --plain times the
+same step with strict stream order.
 """
 from __future__ import annotations
 
@@ -43,7 +48,7 @@ def stack_bytes(stack) -> int:
     return sum(p.numel() + 4 * s.numel() for _, _, _, p, s in stack)
 
 
-def time_stack(stack, bits: int, M: int, reps: int = 20, warmup: int = 3) -> dict:
+def time_stack(stack, bits: int, M: int, reps: int = 20, warmup: int = 3, weights_static: bool = True) -> dict:
     """Capture the token step (all GEMVs of the stack) in a CUDA graph and time it."""
     dev = stack[0][3].device
     gen = torch.Generator(device=dev).manual_seed(4)
@@ -58,7 +63,8 @@ def time_stack(stack, bits: int, M: int, reps: int = 20, warmup: int = 3) -> dic
 
     def step():
         for N, K, g, p, s in stack:
-            qgemm(xs[K], p, s, N, K, bits, g, out=ys[N], workspace=ws.get((N, K, g)))
+            qgemm(xs[K], p, s, N, K, bits, g, out=ys[N], workspace=ws.get((N, K, g)),
+                  weights_static=weights_static)
 
     with torch.cuda.stream(stream):
         step()  # every code path once outside capture
@@ -79,7 +85,7 @@ def time_stack(stack, bits: int, M: int, reps: int = 20, warmup: int = 3) -> dic
     nbytes = stack_bytes(stack)
     del graph
     return {"M": M, "us_per_step": round(us, 1), "gemvs": len(stack), "weight_bytes": nbytes,
-            "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+            "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1), "weights_static": weights_static}
 
 
 def main() -> int:
@@ -89,12 +95,16 @@ def main() -> int:
     ap.add_argument("--M", type=int, nargs="+", default=[1, 4, 16])
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--plain", action="store_true", help="strict stream order (no static-weights flag)")
+    ap.add_argument("--both", action="store_true", help="time both modes")
     a = ap.parse_args()
     stack = build_stack(a.bits, a.group or None, a.layers)
+    modes = (False, True) if a.both else (not a.plain,)
     for M in a.M:
-        r = time_stack(stack, a.bits, M, a.reps)
-        r.update(bits=a.bits, group=a.group or "per-channel", layers=a.layers)
-        print(json.dumps(r), flush=True)
+        for static in modes:
+            r = time_stack(stack, a.bits, M, a.reps, weights_static=static)
+            r.update(bits=a.bits, group=a.group or "per-channel", layers=a.layers)
+            print(json.dumps(r), flush=True)
     return 0
 
 

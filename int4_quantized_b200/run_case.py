@@ -1,12 +1,18 @@
 """Run one library call on a seeded synthetic shape and time it (CUDA events).
 
-    python -m int4_quantized_b200.run_case qgemm N K bits group M [--bf16] [--reps R]
+    python -m int4_quantized_b200.run_case qgemm N K bits group M [--bf16] [--static] [--reps R]
     python -m int4_quantized_b200.run_case qpack N K bits group [--reps R]
 
-W ~ N(0, 0.02) and x ~ N(0, 1) are drawn on the device from a fixed seed. The call is
-made `--warmup` times untimed, then `--reps` times with a CUDA event pair around each; the
-median and the achieved rates are printed as one JSON line (GB/s of the algorithmic bytes:
-payload + scales for qgemm, fp32 input + payload + scales for qpack; TFLOP/s for qgemm).
+W ~ N(0, 0.02) and x ~ N(0, 1) are drawn on the device from a fixed seed. The inputs are
+copied until the copies exceed twice the 126 MB L2 (at most 64 copies), and the calls
+cycle through them, so that every call reads its weights from HBM. `--reps` calls are
+captured in one CUDA graph (launched `--warmup` times untimed, then `--batches` times
+between CUDA events): the per-call time is the batch time over `--reps`, back-to-back
+device time without the host's launch cost. Printed as one JSON line: the median per-call
+time over the batches and the achieved rates (GB/s of the algorithmic bytes: payload +
+scales for qgemm, fp32 input + payload + scales for qpack; TFLOP/s for qgemm).
+`--static` declares the weights static (Q4_QGEMM_WEIGHTS_STATIC), so each call may
+stream its weights while the one before it ends.
 The same command line is what a profiler is pointed at to capture a single kernel.
 """
 from __future__ import annotations
@@ -17,7 +23,9 @@ import statistics
 
 import torch
 
-from . import qgemm, qpack
+from . import qgemm, qgemm_workspace_bytes, qpack
+
+L2_BYTES = 126 * 2 ** 20
 
 
 def main() -> int:
@@ -29,7 +37,9 @@ def main() -> int:
     ap.add_argument("group", type=int)
     ap.add_argument("M", type=int, nargs="?", default=1)
     ap.add_argument("--bf16", action="store_true", help="x in bfloat16 (qgemm)")
-    ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--static", action="store_true", help="weights static (qgemm)")
+    ap.add_argument("--reps", type=int, default=10, help="calls per timed graph")
+    ap.add_argument("--batches", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--seed", type=int, default=0)
     a = ap.parse_args()
@@ -45,27 +55,56 @@ def main() -> int:
         if a.bf16:
             x = x.to(torch.bfloat16)
         y = torch.empty(a.M, a.N, device=dev)
-        call = lambda: qgemm(x, payload, scales, a.N, a.K, a.bits, a.group, out=y)  # noqa: E731
+        ncopy = max(1, min(64, -(-2 * L2_BYTES // pbytes)))
+        P = [payload] + [payload.clone() for _ in range(ncopy - 1)]
+        S = [scales] + [scales.clone() for _ in range(ncopy - 1)]
+        need = qgemm_workspace_bytes(a.M, a.N, a.K, a.bits, a.group, x.dtype)
+        ws = torch.empty(max(256, need), dtype=torch.uint8, device=dev)
+
+        def call(i):
+            j = i % ncopy
+            qgemm(x, P[j], S[j], a.N, a.K, a.bits, a.group, out=y, workspace=ws, weights_static=a.static)
+
         nbytes = pbytes
     else:
-        call = lambda: qpack(w, a.bits, a.group, payload=payload, scales=scales)  # noqa: E731
+        ncopy = max(1, min(64, -(-2 * L2_BYTES // (4 * w.numel() + pbytes))))
+        W = [w] + [w.clone() for _ in range(ncopy - 1)]
+        P = [payload] + [payload.clone() for _ in range(ncopy - 1)]
+        S = [scales] + [scales.clone() for _ in range(ncopy - 1)]
+
+        def call(i):
+            j = i % ncopy
+            qpack(W[j], a.bits, a.group, payload=P[j], scales=S[j])
+
         nbytes = 4 * w.numel() + pbytes
-    for _ in range(a.warmup):
-        call()
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(a.reps):  # every code path once outside capture
+            call(i)
     torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(a.reps):
+            call(i)
     times = []
-    for _ in range(a.reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        call()
-        e1.record()
-        e1.synchronize()
-        times.append(e0.elapsed_time(e1) * 1e3)
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            graph.replay()
+        for _ in range(a.batches):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3 / a.reps)
+    torch.cuda.synchronize()
+    del graph
     us = statistics.median(times)
     out = {"kind": a.kind, "N": a.N, "K": a.K, "bits": a.bits, "group": a.group, "us_median": round(us, 3),
-           "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+           "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1), "copies": ncopy, "calls_per_graph": a.reps}
     if a.kind == "qgemm":
-        out.update(M=a.M, x="bf16" if a.bf16 else "f32", TFLOPs=round(2.0 * a.M * a.N * a.K / (us * 1e-6) / 1e12, 2))
+        out.update(M=a.M, x="bf16" if a.bf16 else "f32", static=a.static,
+                   TFLOPs=round(2.0 * a.M * a.N * a.K / (us * 1e-6) / 1e12, 2))
     print(json.dumps(out), flush=True)
     return 0
 

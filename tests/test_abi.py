@@ -106,6 +106,22 @@ def test_qgemm_workspace_rules(q4):
     assert lib.qgemm(None, 0, 8, None, None, 0, 4096, 4, 128, None, None, 0, None, None) == 0
 
 
+def test_qgemm_ex_flags_and_limits(q4):
+    lib = q4.lib()
+    ok = ctypes.c_void_p(0x100000)
+    need = lib.q4_qgemm_workspace_bytes(8, 4096, 4096, 4, 128, 0)
+    # unknown flag bits are refused before anything else is looked at
+    for flags in (2, 4, 0x80000000):
+        assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need, flags, None, None) == 1
+    # with the static-weights flag the argument rules are those of qgemm
+    assert lib.qgemm_ex(FAKE, 0, 1, FAKE, FAKE, 64, 128, 4, 16, FAKE, None, 0, 1, None, None) == 2
+    assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, 1, None, None) == 5
+    assert lib.qgemm_ex(None, 0, 0, None, None, 4096, 4096, 4, 128, None, None, 0, 1, None, None) == 0
+    # rows of x: at most 65535 chunks of 16
+    assert q4.qgemm_workspace_bytes(65535 * 16, 256, 1024, 4, 128) > 0
+    assert lib.qgemm(FAKE, 0, 65535 * 16 + 1, FAKE, FAKE, 256, 1024, 4, 128, FAKE, ok, 1 << 40, None, None) == 2
+
+
 def test_workspace_is_a_pure_function_of_the_problem(q4):
     for M in (1, 4, 8, 16, 40, 300, 2048):
         a = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)
