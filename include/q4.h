@@ -212,6 +212,53 @@ Q4_API q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uin
                 const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
                 uint32_t *status_word, void *stream);
 
+/*
+ * ---- GPTQ host quantizer ("Huit bits, puis quatre", section "Arrondir mieux :
+ * GPTQ"). Host code, fp64; every pointer below is HOST memory owned by the
+ * caller. The result is a payload + scales pair in exactly the format of
+ * qpack, read by qdequant and qgemm unchanged: the same codes, chosen so that
+ * the layer's output x W'^T moves as little as possible on typical inputs x.
+ */
+
+/*
+ * q4_gptq_hessian -- H += sum over the rows r of x: x[r]^T x[r], in fp64.
+ *   x  [rows][K] fp32 calibration inputs of the layer (row-major)
+ *   H  [K][K] fp64, accumulated in place (zero it before the first batch)
+ *   threads  worker threads (0 = all hardware threads); each owns rows of H,
+ *            so the result does not depend on it
+ * Errors: Q4_ERR_ARG (shapes, null), Q4_ERR_NONFINITE (x holds NaN or Inf;
+ * H is left untouched).
+ */
+Q4_API q4_status q4_gptq_hessian(const float *x, int64_t rows, int64_t K, double *H, int threads);
+
+/*
+ * q4_gptq_prepare -- U, upper triangular, with (H + damp * mean(diag H) * I)^-1
+ * = U^T U. The page adds damp = 0.01. O(K^3) on one thread.
+ *   H  [K][K] fp64 (symmetric; the mean of its two triangles is used)
+ *   U  [K][K] fp64 out, zeros below the diagonal
+ * Errors: Q4_ERR_ARG (null, K < 1, damp < 0, mean(diag H) <= 0, or the damped
+ * H is not positive definite).
+ */
+Q4_API q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U);
+
+/*
+ * q4_gptq_quantize -- the payload and scales of W [N][K] (fp32, row-major,
+ * groups of `group` consecutive weights along K) by GPTQ: the columns k are
+ * quantized in order; the error of column k, (w - code * scale) / U[k][k], is
+ * taken off each later column j times U[k][j]; a group's scales are set, by
+ * the qpack rule, from the corrected weights when its first column is reached.
+ *   U        from q4_gptq_prepare (any upper triangular U with a nonzero
+ *            diagonal is accepted; a diagonal U gives exactly qpack's result)
+ *   payload  out, q4_payload_bytes(N, K, bits) bytes
+ *   scales   out, N * K / group floats
+ *   threads  worker threads over rows (0 = all); the result does not depend on it
+ * Cost: N * K^2 / 2 multiply-subtracts. Requirements: bits 4 or 8, group
+ * divides K, N * K even for int4.
+ * Errors: Q4_ERR_ARG, Q4_ERR_NONFINITE (W holds NaN or Inf; outputs untouched).
+ */
+Q4_API q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U, int bits,
+                int64_t group, uint8_t *payload, float *scales, int threads);
+
 #ifdef __cplusplus
 }
 #endif

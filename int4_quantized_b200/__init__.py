@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "Q4Error", "lib", "lib_path", "payload_bytes", "num_scales", "qgemm_workspace_bytes",
-    "qpack", "qdequant", "qgemm", "qgemm_noalloc", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
+    "qpack", "qdequant", "qgemm", "qgemm_noalloc", "gptq_hessian", "gptq_prepare", "gptq_quantize", "gptq_pack", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
     "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_ERR_SCRATCH_LIMIT", "Q4_X_F32", "Q4_X_BF16", "Q4_QGEMM_WEIGHTS_STATIC", "STATUS_NONFINITE", "STATUS_TIMEOUT",
 ]
 
@@ -79,6 +79,12 @@ def lib() -> ctypes.CDLL:
                 L.qgemm_ex.restype = i32
                 L.qgemm_noalloc.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, vp]
                 L.qgemm_noalloc.restype = i32
+                L.q4_gptq_hessian.argtypes = [vp, i64, i64, vp, i32]
+                L.q4_gptq_hessian.restype = i32
+                L.q4_gptq_prepare.argtypes = [vp, i64, ctypes.c_double, vp]
+                L.q4_gptq_prepare.restype = i32
+                L.q4_gptq_quantize.argtypes = [vp, i64, i64, vp, i32, i64, vp, vp, i32]
+                L.q4_gptq_quantize.restype = i32
                 _lib = L
     return _lib
 
@@ -226,3 +232,68 @@ def qgemm_noalloc(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, 
         _check(lib().qgemm_noalloc(_ptr(x), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group,
                                    _ptr(out), _ptr(status), _stream(x.device)), "qgemm_noalloc")
     return out
+
+
+# ---- GPTQ host quantizer (host arrays; the computation runs in libq4's C++ code) ----------
+
+def _host(a, dtype, name):
+    import numpy as np
+
+    if isinstance(a, torch.Tensor):
+        if a.is_cuda:
+            raise TypeError(f"{name} must be host memory (a NumPy array or a CPU tensor)")
+        a = a.numpy()
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"{name} must be {np.dtype(dtype).name}, got {a.dtype}")
+    return a
+
+
+def gptq_hessian(x, H=None, threads: int = 0):
+    """H += x^T x in fp64 for calibration inputs x [rows, K] float32 (H new when None)."""
+    import numpy as np
+
+    x = _host(x, np.float32, "x")
+    rows, K = x.shape
+    if H is None:
+        H = np.zeros((K, K), np.float64)
+    elif not (isinstance(H, np.ndarray) and H.dtype == np.float64 and H.shape == (K, K) and H.flags.c_contiguous):
+        raise TypeError("H must be a C-contiguous float64 [K, K] NumPy array")
+    _check(lib().q4_gptq_hessian(x.ctypes.data_as(ctypes.c_void_p), rows, K, H.ctypes.data_as(ctypes.c_void_p),
+                                 threads), "gptq_hessian")
+    return H
+
+
+def gptq_prepare(H, damp: float = 0.01):
+    """U (upper, fp64) with (H + damp * mean(diag H) * I)^-1 = U^T U."""
+    import numpy as np
+
+    H = _host(H, np.float64, "H")
+    K = H.shape[0]
+    U = np.empty((K, K), np.float64)
+    _check(lib().q4_gptq_prepare(H.ctypes.data_as(ctypes.c_void_p), K, damp, U.ctypes.data_as(ctypes.c_void_p)),
+           "gptq_prepare")
+    return U
+
+
+def gptq_quantize(w, U, bits: int, group: int, threads: int = 0):
+    """(payload uint8, scales float32) of W [N, K] float32 by GPTQ, in qpack's format."""
+    import numpy as np
+
+    w = _host(w, np.float32, "w")
+    U = _host(U, np.float64, "U")
+    N, K = w.shape
+    if U.shape != (K, K):
+        raise ValueError("U must be [K, K]")
+    payload = np.empty(N * K * bits // 8, np.uint8)
+    scales = np.empty(N * K // group if group > 0 and K % group == 0 else 0, np.float32)
+    _check(lib().q4_gptq_quantize(w.ctypes.data_as(ctypes.c_void_p), N, K, U.ctypes.data_as(ctypes.c_void_p), bits,
+                                  group, payload.ctypes.data_as(ctypes.c_void_p),
+                                  scales.ctypes.data_as(ctypes.c_void_p), threads), "gptq_quantize")
+    return payload, scales
+
+
+def gptq_pack(w, x, bits: int, group: int, damp: float = 0.01, threads: int = 0):
+    """GPTQ end to end on the host: H from calibration inputs x [rows, K], then the codes."""
+    H = gptq_hessian(x, threads=threads)
+    return gptq_quantize(w, gptq_prepare(H, damp), bits, group, threads)

@@ -2,7 +2,8 @@
 
 Run as ``python -m int4_quantized_b200._build`` or through ``__graft_entry__.build()``.
 nvcc cross-compiles without a GPU. The kernels rely on IEEE division and denormals, so
-there is no --use_fast_math and -prec-div/-ftz are pinned explicitly.
+there is no --use_fast_math and -prec-div/-ftz are pinned explicitly; host code (the GPTQ
+quantizer in csrc/gptq.cpp) is built without floating-point contraction.
 """
 from __future__ import annotations
 
@@ -14,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libq4.so")
-SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
+SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) + glob.glob(os.path.join(HERE, "csrc", "*.cpp")))
 DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + \
     sorted(glob.glob(os.path.join(HERE, "csrc", "*.h"))) + [os.path.join(ROOT, "include", "q4.h")]
 
@@ -22,7 +23,7 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "-prec-div=true", "-prec-sqrt=true", "-ftz=false",
-    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden,-ffp-contract=off",
     "-shared", "-cudart", "static",
     "-I", os.path.join(ROOT, "include"),
 ]

@@ -1,0 +1,172 @@
+// gptq.cpp -- the GPTQ host quantizer (host code, fp64): codes chosen to keep a layer's
+// output, in the same payload format as qpack ("Huit bits, puis quatre", section "Arrondir
+// mieux : GPTQ").
+//
+// With H = sum over calibration samples of x^T x ([K, K]) and U the upper triangular
+// factor of (H + damping)^-1 = U^T U, the input components k (the columns of W [N, K])
+// are quantized in order; the error of column k, divided by U[k][k], is taken off every
+// later column j in proportion to U[k][j]. A group's scale is fixed when its first column
+// is reached, from the weights corrected so far, by the rounding rule of qpack (scale =
+// max|w| / qmax in fp32, 0 -> 1; code = clip(rint(w / scale)) with an IEEE fp32 divide).
+// Each output row only ever reads its own weights, so rows run on separate threads; the
+// operations on every weight are those of the definition, in its order.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "../../include/q4.h"
+
+namespace {
+
+inline bool finite_all(const float *p, int64_t n) {
+    for (int64_t i = 0; i < n; ++i)
+        if (!std::isfinite(p[i])) return false;
+    return true;
+}
+
+inline int qmax_of(int bits) { return bits == 4 ? 7 : 127; }
+
+// Run f(lo, hi) over [0, n) split into contiguous parts, one per thread.
+template <typename F>
+void parallel_rows(int64_t n, int threads, F f) {
+    int t = threads > 0 ? threads : (int)std::thread::hardware_concurrency();
+    if (t < 1) t = 1;
+    if (t > n) t = (int)std::max<int64_t>(n, 1);
+    if (t == 1) {
+        f((int64_t)0, n);
+        return;
+    }
+    std::vector<std::thread> pool;
+    for (int i = 0; i < t; ++i) {
+        const int64_t lo = n * i / t, hi = n * (i + 1) / t;
+        pool.emplace_back([=] { f(lo, hi); });
+    }
+    for (auto &th : pool) th.join();
+}
+
+// In place lower Cholesky factor of the symmetric [K, K] matrix A (A = L L^T); the strict
+// upper triangle is set to zero. False when A is not positive definite.
+bool cholesky_lower(std::vector<double> &A, int64_t K) {
+    for (int64_t j = 0; j < K; ++j) {
+        double *aj = &A[j * K];
+        double d = aj[j];
+        for (int64_t p = 0; p < j; ++p) d -= aj[p] * aj[p];
+        if (!(d > 0.0) || !std::isfinite(d)) return false;
+        const double ljj = std::sqrt(d);
+        aj[j] = ljj;
+        for (int64_t i = j + 1; i < K; ++i) {
+            double *ai = &A[i * K];
+            double s = ai[j];
+            for (int64_t p = 0; p < j; ++p) s -= ai[p] * aj[p];
+            ai[j] = s / ljj;
+        }
+        for (int64_t i = j + 1; i < K; ++i) aj[i] = 0.0;
+    }
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+q4_status q4_gptq_hessian(const float *x, int64_t rows, int64_t K, double *H, int threads) {
+    if (rows < 0 || K < 1 || !H || (rows > 0 && !x)) return Q4_ERR_ARG;
+    if (!finite_all(x, rows * K)) return Q4_ERR_NONFINITE;
+    // thread i owns rows [lo, hi) of H; samples are added in order
+    parallel_rows(K, threads, [&](int64_t lo, int64_t hi) {
+        for (int64_t r = 0; r < rows; ++r) {
+            const float *xr = x + r * K;
+            for (int64_t i = lo; i < hi; ++i) {
+                const double xi = (double)xr[i];
+                double *hi_row = H + i * K;
+                for (int64_t j = 0; j < K; ++j) hi_row[j] += xi * (double)xr[j];
+            }
+        }
+    });
+    return Q4_OK;
+}
+
+q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U) {
+    if (!H || !U || K < 1 || !(damp >= 0.0)) return Q4_ERR_ARG;
+    double mean = 0.0;
+    for (int64_t i = 0; i < K; ++i) mean += H[i * K + i];
+    mean /= (double)K;
+    if (!(mean > 0.0) || !std::isfinite(mean)) return Q4_ERR_ARG;
+    // (H + d I)^-1 = U^T U with U upper  <=>  H + d I = V V^T with V = U^-1 upper. With J the
+    // order reversal, J (H + d I) J = (J V J)(J V J)^T is a lower Cholesky factorisation, so
+    // U = J L^-1 J for L = chol(J (H + d I) J).
+    std::vector<double> A((size_t)(K * K));
+    for (int64_t i = 0; i < K; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            const double h = 0.5 * (H[i * K + j] + H[j * K + i]);
+            A[(K - 1 - i) * K + (K - 1 - j)] = h + (i == j ? damp * mean : 0.0);
+        }
+    if (!cholesky_lower(A, K)) return Q4_ERR_ARG;
+    // column c of L^-1 by forward substitution (x_c = 1 / L[c][c]; x_i for i > c), written
+    // straight into U[K-1-i][K-1-c]
+    std::vector<double> x((size_t)K);
+    std::fill(U, U + K * K, 0.0);
+    for (int64_t c = 0; c < K; ++c) {
+        x[c] = 1.0 / A[c * K + c];
+        for (int64_t i = c + 1; i < K; ++i) {
+            const double *li = &A[i * K];
+            double s = 0.0;
+            for (int64_t p = c; p < i; ++p) s += li[p] * x[p];
+            x[i] = -s / li[i];
+        }
+        for (int64_t i = c; i < K; ++i) U[(K - 1 - i) * K + (K - 1 - c)] = x[i];
+    }
+    return Q4_OK;
+}
+
+q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U, int bits, int64_t group,
+                           uint8_t *payload, float *scales, int threads) {
+    if (bits != 4 && bits != 8) return Q4_ERR_ARG;
+    if (N < 0 || K < 1 || group < 1 || K % group != 0) return Q4_ERR_ARG;
+    if (bits == 4 && (N * K) % 2 != 0) return Q4_ERR_ARG;
+    if (N == 0) return Q4_OK;
+    if (!w || !U || !payload || !scales) return Q4_ERR_ARG;
+    for (int64_t k = 0; k < K; ++k)
+        if (!(U[k * K + k] != 0.0) || !std::isfinite(U[k * K + k])) return Q4_ERR_ARG;
+    if (!finite_all(w, N * K)) return Q4_ERR_NONFINITE;
+    const int qmax = qmax_of(bits);
+    const int64_t spr = K / group;
+    std::vector<int8_t> codes((size_t)(N * K));
+    parallel_rows(N, threads, [&](int64_t lo, int64_t hi) {
+        std::vector<double> W((size_t)K);
+        for (int64_t n = lo; n < hi; ++n) {
+            for (int64_t k = 0; k < K; ++k) W[k] = (double)w[n * K + k];
+            float s = 1.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                if (k % group == 0) {
+                    float a = 0.0f;
+                    for (int64_t j = k; j < k + group; ++j) a = std::max(a, std::fabs((float)W[j]));
+                    s = a / (float)qmax;
+                    if (s == 0.0f) s = 1.0f;
+                    scales[n * spr + k / group] = s;
+                }
+                const float t = (float)W[k] / s;
+                float c = std::nearbyint(t);
+                c = std::min(std::max(c, (float)-qmax), (float)qmax);
+                codes[n * K + k] = (int8_t)c;
+                const double wq = (double)(c * s);
+                const double err = (W[k] - wq) / U[k * K + k];
+                const double *uk = U + k * K;
+                for (int64_t j = k + 1; j < K; ++j) W[j] -= err * uk[j];
+            }
+        }
+    });
+    const int64_t n = N * K;
+    if (bits == 8) {
+        std::memcpy(payload, codes.data(), (size_t)n);
+    } else {
+        for (int64_t t = 0; t < n / 2; ++t)
+            payload[t] = (uint8_t)((codes[2 * t] + 8) | ((codes[2 * t + 1] + 8) << 4));
+    }
+    return Q4_OK;
+}
+
+}  // extern "C"
