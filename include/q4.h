@@ -118,8 +118,10 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
  * fragment order (4 bytes per element of x, rows padded to pairs and 16-row
  * chunks) plus one exponent per row of x and block of up to 1024 k. One row
  * of x needs none (0) when each CTA's share of K fits on chip, which holds up
- * to K = 8192 per CTA. Same arguments as qgemm. Returns 0 for arguments qgemm
- * rejects. Depends only on the arguments, not on the device.
+ * to K = 8192 per CTA. Groups of whole rows (group a multiple of K) add N
+ * floats, rounded up to 256 bytes, at the start: their scales spread to one
+ * per row. Same arguments as qgemm. Returns 0 for arguments qgemm rejects.
+ * Depends only on the arguments, not on the device.
  */
 Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt);
@@ -146,10 +148,15 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * (rows of x in chunks of 16). bf16 x with M >= 64: the tensor-core GEMM.
  * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
  * finite inputs (y_exact = the fp64 sum).
- * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0, group divides K and
- * group % 32 == 0 (per-channel scales are group = K); N, K <= 2^30 and
- * M <= 1048560 (65535 chunks of 16 rows). M, N >= 0; M == 0 or N == 0
- * enqueues nothing.
+ * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0; group divides K with
+ * group % 32 == 0 (per-channel scales are group = K), or group is a multiple
+ * of K (groups of whole rows, down to one scale for the whole matrix, the
+ * INT4_TENSOR format of the "量化推理：INT8/INT4 ..." page; N must then be a
+ * multiple of group / K, else Q4_ERR_ARG). Groups of whole rows are spread to
+ * one scale per row in the workspace by a first kernel, which the fused path
+ * then reads (Q4_QGEMM_WEIGHTS_STATIC has no effect on such calls).
+ * N, K <= 2^30 and M <= 1048560 (65535 chunks of 16 rows). M, N >= 0;
+ * M == 0 or N == 0 enqueues nothing.
  * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
  * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
  */

@@ -9,6 +9,12 @@
 
 #include "kernels.h"
 
+namespace q4 {
+// rowscale.cu: out[n] = scales[n / rows_per_scale] for n < N
+cudaError_t launch_expand_row_scales(const float *scales, int64_t rows_per_scale, int64_t N, float *out,
+                                     cudaStream_t st);
+}  // namespace q4
+
 namespace {
 
 // qgemm's task split is planned for a full B200 (148 SMs) whatever device runs it, so
@@ -39,15 +45,38 @@ q4_status check_format(int64_t rows, int64_t cols, int bits, int64_t group, int6
     return Q4_OK;
 }
 
-// Path selection for qgemm: returns Q4_OK and fills the plan, or the reason it cannot run.
-q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q4_xdtype xt,
-                     q4::GemvPlan *pl) {
+inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Path selection and workspace layout of one qgemm call.
+struct QgemmPlan {
+    q4::GemvPlan gemv;    // the fused GEMV plan (for the row-scale group when rps > 1)
+    int64_t group;        // group the kernels see: the caller's, or K for groups of whole rows
+    int64_t rps;          // rows per scale when the group spans whole rows, else 1
+    bool prefill;         // bf16 x, M >= 64: the tensor-core GEMM
+    size_t scale_bytes;   // expanded per-row scales at the start of the workspace (rps > 1)
+    size_t total_bytes;   // workspace the call needs
+};
+
+// Returns Q4_OK and fills the plan, or the reason the call cannot run. Groups either divide
+// K, or are whole multiples of K (c rows share a scale; their scales are first expanded to
+// one per row in the workspace).
+q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q4_xdtype xt, QgemmPlan *p) {
     if (bits != 4 && bits != 8) return Q4_ERR_ARG;
     if (M < 0 || N < 0 || K < 1 || group < 1) return Q4_ERR_ARG;
     if (xt != Q4_X_F32 && xt != Q4_X_BF16) return Q4_ERR_ARG;
-    if (K % group != 0) return Q4_ERR_UNSUPPORTED;
-    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, group, kPlanSMs, pl))
+    p->group = group;
+    p->rps = 1;
+    if (K % group != 0) {
+        if (group % K != 0) return Q4_ERR_UNSUPPORTED;
+        p->rps = group / K;
+        if (N % p->rps != 0) return Q4_ERR_ARG;  // no [N][K] matrix has such groups
+        p->group = K;
+    }
+    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, p->group, kPlanSMs, &p->gemv))
         return Q4_ERR_UNSUPPORTED;
+    p->prefill = q4::prefill_supported(M, N, K, bits, p->group, xt == Q4_X_BF16);
+    p->scale_bytes = p->rps > 1 ? align256((size_t)N * 4) : 0;
+    p->total_bytes = p->scale_bytes + (p->prefill ? 0 : p->gemv.bytes);
     return Q4_OK;
 }
 
@@ -131,10 +160,9 @@ q4_status qdequant(const uint8_t *payload, const float *scales, int64_t rows, in
 
 size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt) {
-    q4::GemvPlan pl;
-    if (plan_qgemm(M, N, K, bits, group, xt, &pl) != Q4_OK) return 0;
-    if (q4::prefill_supported(M, N, K, bits, group, xt == Q4_X_BF16)) return 0;
-    return pl.bytes;
+    QgemmPlan p;
+    if (plan_qgemm(M, N, K, bits, group, xt, &p) != Q4_OK) return 0;
+    return p.total_bytes;
 }
 
 q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
@@ -142,22 +170,32 @@ q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payloa
                    void *workspace, size_t workspace_bytes, uint32_t flags, uint32_t *status_word,
                    void *stream) {
     if (flags & ~(uint32_t)Q4_QGEMM_WEIGHTS_STATIC) return Q4_ERR_ARG;
-    q4::GemvPlan pl;
-    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &pl);
+    QgemmPlan p;
+    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &p);
     if (st != Q4_OK) return st;
     if (M == 0 || N == 0) return Q4_OK;
     if (!x || !payload || !scales || !y) return Q4_ERR_ARG;
     if ((uintptr_t)payload % 16 || (uintptr_t)x % 16) return Q4_ERR_UNSUPPORTED;
-    if (q4::prefill_supported(M, N, K, bits, group, xt == Q4_X_BF16)) {
-        cudaError_t e = q4::launch_prefill(x, M, payload, scales, N, K, bits, group, y, status_word,
-                                           device_sms(), as_stream(stream));
-        return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    if ((!p.prefill || p.total_bytes > 0) && (uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
+    if (p.total_bytes > 0 && (!workspace || workspace_bytes < p.total_bytes)) return Q4_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    const float *sc = scales;
+    bool early = (flags & Q4_QGEMM_WEIGHTS_STATIC) != 0;
+    if (p.rps > 1) {
+        // one scale per row, written by the kernel just before: no early start
+        float *rs = static_cast<float *>(workspace);
+        if (q4::launch_expand_row_scales(scales, p.rps, N, rs, s) != cudaSuccess) return Q4_ERR_CUDA;
+        sc = rs;
+        early = false;
     }
-    if ((uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
-    if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return Q4_ERR_WORKSPACE;
-    cudaError_t e = q4::launch_gemv(pl, x, xt == Q4_X_BF16, M, payload, scales, N, K, group, y,
-                                    workspace, status_word, (flags & Q4_QGEMM_WEIGHTS_STATIC) != 0,
-                                    as_stream(stream));
+    cudaError_t e;
+    if (p.prefill) {
+        e = q4::launch_prefill(x, M, payload, sc, N, K, bits, p.group, y, status_word, device_sms(), s);
+    } else {
+        void *ws = p.gemv.bytes ? static_cast<char *>(workspace) + p.scale_bytes : nullptr;
+        e = q4::launch_gemv(p.gemv, x, xt == Q4_X_BF16, M, payload, sc, N, K, p.group, y, ws, status_word, early,
+                            s);
+    }
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
@@ -171,11 +209,11 @@ q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
 q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
                         const float *scales, int64_t N, int64_t K, int bits, int64_t group,
                         float *y, uint32_t *status_word, void *stream) {
-    q4::GemvPlan pl;
-    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &pl);
+    QgemmPlan p;
+    q4_status st = plan_qgemm(M, N, K, bits, group, xt, &p);
     if (st != Q4_OK) return st;
     if (M == 0 || N == 0) return Q4_OK;
-    if (pl.bytes > kNoAllocBytes) return Q4_ERR_SCRATCH_LIMIT;
+    if (p.total_bytes > kNoAllocBytes) return Q4_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
     st = noalloc_scratch(&scratch);
     if (st != Q4_OK) return st;

@@ -122,6 +122,26 @@ def test_qgemm_ex_flags_and_limits(q4):
     assert lib.qgemm(FAKE, 0, 65535 * 16 + 1, FAKE, FAKE, 256, 1024, 4, 128, FAKE, ok, 1 << 40, None, None) == 2
 
 
+def test_groups_of_whole_rows(q4):
+    import torch
+
+    lib = q4.lib()
+    N, K = 64, 256
+    # one scale for the whole matrix, and groups of 2 and 4 rows: N floats of spread scales
+    for g in (N * K, 2 * K, 4 * K):
+        assert q4.qgemm_workspace_bytes(1, N, K, 4, g) == 256
+        assert q4.qgemm_workspace_bytes(300, N, K, 4, g, torch.bfloat16) == 256  # the GEMM needs only those
+        assert q4.qgemm_workspace_bytes(8, N, K, 8, g) == 256 + q4.qgemm_workspace_bytes(8, N, K, 8, K)
+    assert q4.qgemm_workspace_bytes(1, 1000, K, 4, K * 1000) == 4096
+    # groups that neither divide K nor are whole rows; N not a multiple of the rows per group
+    ok = ctypes.c_void_p(0x100000)
+    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, 3 * K // 2, FAKE, ok, 1 << 20, None, None) == 2
+    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, 63, K, 4, 2 * K, FAKE, ok, 1 << 20, None, None) == 1
+    # the spread scales must fit in the workspace
+    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, N * K, FAKE, ok, 255, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, N * K, FAKE, None, 0, None, None) == 5
+
+
 def test_workspace_is_a_pure_function_of_the_problem(q4):
     for M in (1, 4, 8, 16, 40, 300, 2048):
         a = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)

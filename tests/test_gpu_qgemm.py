@@ -213,3 +213,36 @@ def test_deterministic(q4):
     a = run_gpu(q4, x, payload, scales, 4096, 4096, 4, 128)
     b = run_gpu(q4, x, payload, scales, 4096, 4096, 4, 128)
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rows_per_group", ["all", 2, 8])
+@pytest.mark.parametrize("M,bf16", [(1, False), (5, False), (96, True)])
+def test_groups_of_whole_rows(q4, bits, rows_per_group, M, bf16):
+    # one scale for the whole matrix (the INT4_TENSOR format) or one per few rows
+    import torch
+
+    N, K = 320, 512
+    g = N * K if rows_per_group == "all" else rows_per_group * K
+    rng = np.random.default_rng(M * 10 + bits)
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    w.reshape(-1)[rng.choice(N * K, 40, replace=False)] *= 20
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    payload, scales, _ = oracle.pack(w, bits, g)
+    assert scales.size == N * K // g
+    xin = torch.from_numpy(x).to(torch.bfloat16).float().numpy() if bf16 else x
+    xt = torch.from_numpy(x).cuda()
+    if bf16:
+        xt = xt.to(torch.bfloat16)
+    P, S = torch.from_numpy(payload).cuda(), torch.from_numpy(scales).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.qgemm(xt, P, S, N, K, bits, g, status=status)
+    y2 = q4.qgemm(xt, P, S, N, K, bits, g, status=status, weights_static=True)
+    y3 = torch.empty_like(y)
+    q4.qgemm_noalloc(xt, P, S, N, K, bits, g, y3, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    yref, bound = oracle.qgemm(xin, payload, scales, N, K, bits, g)
+    check(y.cpu().numpy(), yref, bound, f"int{bits} g{g} M{M}")
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+    assert torch.equal(y.view(torch.int32), y3.view(torch.int32))
