@@ -141,9 +141,10 @@ Q4_DEVINL float scale_of_f(float absmax) {
 // float4 at 4 * (32 u + l), so every load instruction reads 512 contiguous bytes. A group
 // of G <= 128 lies inside one load (G/4 lanes, shuffle reduction); a larger group spans
 // G/128 loads of the whole warp. Packed bytes are transposed through shared memory so
-// that each lane writes one (int4) or two (int8) 128-bit stores.
+// that each lane writes one (int4) or two (int8) 128-bit stores. Registers are capped
+// for four CTAs (32 warps) per SM: more chunks in flight per SM to cover the load latency.
 template <int BITS, int G>
-__global__ void __launch_bounds__(256, 2) qpack_chunk(const float *__restrict__ w, int64_t nchunks,
+__global__ void __launch_bounds__(256, 4) qpack_chunk(const float *__restrict__ w, int64_t nchunks,
                                                       uint8_t *__restrict__ payload,
                                                       float *__restrict__ scales,
                                                       uint32_t *__restrict__ status) {
