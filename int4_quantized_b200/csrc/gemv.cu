@@ -428,6 +428,12 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         }
         fence_barrier_init();
     }
+    if constexpr (INK) {
+        // block maxima of the on-chip digits, zeroed before the barrier that publishes the
+        // mbarriers. A CTA's digits fit in kFragCap: at most 32 int4 stages (k-blocks of one
+        // or more) or 64 int8 stages (k-blocks of two or more), so at most 33 local k-blocks.
+        for (int i = threadIdx.x; i < kMaxLocalBlocks; i += blockDim.x) mx_sh[i] = 0;
+    }
     __syncthreads();
 
     // groups [gA, gA + ng) touched by k-block eb inside this CTA's range
@@ -527,9 +533,6 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             // first payload tiles are in flight; x may be the output of the kernel before
             // this one (a no-op unless this grid was launched as a dependent)
             grid_dep_wait();
-            const int nlb = nst > 0 ? (st_hi - 1) / a.ebs - eb_first + 1 : 0;
-            for (int i = ct; i < nlb; i += kConsumerThreads) mx_sh[i] = 0;
-            named_barrier_sync(1, kConsumerThreads);
             const int k_lo = st_lo * STAGEK, k_hi = min(st_hi * STAGEK, a.K);
             const int nu = max(k_hi - k_lo, 0) / 8;
             constexpr int R = kFragCap / 4 / 8 / kConsumerThreads;  // units per thread (4)
@@ -811,6 +814,9 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;
+    // chunks of 9-16 rows of x (NB == 8) ignore the flag: their early start was measured
+    // slower (a Llama-7B-shaped decode step at M = 16: 4.93 ms against 4.81 ms)
+    if (NB > 4) early = false;
     if constexpr (!INK) {
         cudaLaunchConfig_t pc = {};
         pc.gridDim = dim3(pl.n_eb, pl.nmc);
