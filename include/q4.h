@@ -240,13 +240,14 @@ Q4_API q4_status q4_gptq_hessian(const float *x, int64_t rows, int64_t K, double
 
 /*
  * q4_gptq_prepare -- U, upper triangular, with (H + damp * mean(diag H) * I)^-1
- * = U^T U. The page adds damp = 0.01. O(K^3) on one thread.
+ * = U^T U. The page adds damp = 0.01. O(K^3), split over threads.
  *   H  [K][K] fp64 (symmetric; the mean of its two triangles is used)
  *   U  [K][K] fp64 out, zeros below the diagonal
+ *   threads  worker threads (0 = all hardware threads); U does not depend on it
  * Errors: Q4_ERR_ARG (null, K < 1, damp < 0, mean(diag H) <= 0, or the damped
  * H is not positive definite).
  */
-Q4_API q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U);
+Q4_API q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U, int threads);
 
 /*
  * q4_gptq_quantize -- the payload and scales of W [N][K] (fp32, row-major,

@@ -81,7 +81,7 @@ def lib() -> ctypes.CDLL:
                 L.qgemm_noalloc.restype = i32
                 L.q4_gptq_hessian.argtypes = [vp, i64, i64, vp, i32]
                 L.q4_gptq_hessian.restype = i32
-                L.q4_gptq_prepare.argtypes = [vp, i64, ctypes.c_double, vp]
+                L.q4_gptq_prepare.argtypes = [vp, i64, ctypes.c_double, vp, i32]
                 L.q4_gptq_prepare.restype = i32
                 L.q4_gptq_quantize.argtypes = [vp, i64, i64, vp, i32, i64, vp, vp, i32]
                 L.q4_gptq_quantize.restype = i32
@@ -264,15 +264,15 @@ def gptq_hessian(x, H=None, threads: int = 0):
     return H
 
 
-def gptq_prepare(H, damp: float = 0.01):
+def gptq_prepare(H, damp: float = 0.01, threads: int = 0):
     """U (upper, fp64) with (H + damp * mean(diag H) * I)^-1 = U^T U."""
     import numpy as np
 
     H = _host(H, np.float64, "H")
     K = H.shape[0]
     U = np.empty((K, K), np.float64)
-    _check(lib().q4_gptq_prepare(H.ctypes.data_as(ctypes.c_void_p), K, damp, U.ctypes.data_as(ctypes.c_void_p)),
-           "gptq_prepare")
+    _check(lib().q4_gptq_prepare(H.ctypes.data_as(ctypes.c_void_p), K, damp, U.ctypes.data_as(ctypes.c_void_p),
+                                 threads), "gptq_prepare")
     return U
 
 
@@ -296,4 +296,4 @@ def gptq_quantize(w, U, bits: int, group: int, threads: int = 0):
 def gptq_pack(w, x, bits: int, group: int, damp: float = 0.01, threads: int = 0):
     """GPTQ end to end on the host: H from calibration inputs x [rows, K], then the codes."""
     H = gptq_hessian(x, threads=threads)
-    return gptq_quantize(w, gptq_prepare(H, damp), bits, group, threads)
+    return gptq_quantize(w, gptq_prepare(H, damp, threads), bits, group, threads)

@@ -12,8 +12,10 @@
 // operations on every weight are those of the definition, in its order.
 #include <algorithm>
 #include <cmath>
+#include <condition_variable>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -47,23 +49,79 @@ void parallel_rows(int64_t n, int threads, F f) {
     for (auto &th : pool) th.join();
 }
 
-// In place lower Cholesky factor of the symmetric [K, K] matrix A (A = L L^T); the strict
-// upper triangle is set to zero. False when A is not positive definite.
-bool cholesky_lower(std::vector<double> &A, int64_t K) {
-    for (int64_t j = 0; j < K; ++j) {
-        double *aj = &A[j * K];
-        double d = aj[j];
-        for (int64_t p = 0; p < j; ++p) d -= aj[p] * aj[p];
-        if (!(d > 0.0) || !std::isfinite(d)) return false;
-        const double ljj = std::sqrt(d);
-        aj[j] = ljj;
-        for (int64_t i = j + 1; i < K; ++i) {
-            double *ai = &A[i * K];
-            double s = ai[j];
-            for (int64_t p = 0; p < j; ++p) s -= ai[p] * aj[p];
-            ai[j] = s / ljj;
+int thread_count(int threads, int64_t work_items) {
+    int t = threads > 0 ? threads : (int)std::thread::hardware_concurrency();
+    if (t < 1) t = 1;
+    if (t > work_items) t = (int)std::max<int64_t>(work_items, 1);
+    return t;
+}
+
+// A reusable barrier for a fixed set of threads (C++17 has none).
+class Barrier {
+  public:
+    explicit Barrier(int n) : n_(n) {}
+    void wait() {
+        std::unique_lock<std::mutex> lk(mu_);
+        const uint64_t gen = gen_;
+        if (++count_ == n_) {
+            count_ = 0;
+            ++gen_;
+            cv_.notify_all();
+        } else {
+            cv_.wait(lk, [&] { return gen_ != gen; });
         }
-        for (int64_t i = j + 1; i < K; ++i) aj[i] = 0.0;
+    }
+
+  private:
+    std::mutex mu_;
+    std::condition_variable cv_;
+    int n_, count_ = 0;
+    uint64_t gen_ = 0;
+};
+
+// In place lower Cholesky factor of the symmetric [K, K] matrix A (A = L L^T), column by
+// column; the strict upper triangle is set to zero. False when A is not positive definite.
+// Rows below the diagonal are shared cyclically among the threads, one barrier per column;
+// every thread forms the column's diagonal itself (the same operations on the same
+// values), so the factor is the same for any thread count.
+bool cholesky_lower(std::vector<double> &A, int64_t K, int threads) {
+    const int T = thread_count(threads, K / 64);
+    std::vector<double> diag((size_t)K);
+    bool ok = true;
+    Barrier bar(T);
+    auto work = [&](int tid) {
+        for (int64_t j = 0; j < K; ++j) {
+            const double *aj = &A[j * K];
+            double d = aj[j];
+            for (int64_t p = 0; p < j; ++p) d -= aj[p] * aj[p];
+            const bool pd = d > 0.0 && std::isfinite(d);
+            if (!pd) {
+                if (tid == 0) ok = false;
+                return;  // every thread sees the same d and leaves at the same column
+            }
+            const double ljj = std::sqrt(d);
+            if (j % T == tid) diag[j] = ljj;
+            int64_t i0 = j + 1 + ((tid - (j + 1)) % T + T) % T;  // first row > j owned by tid
+            for (int64_t i = i0; i < K; i += T) {
+                double *ai = &A[i * K];
+                double s = ai[j];
+                for (int64_t p = 0; p < j; ++p) s -= ai[p] * aj[p];
+                ai[j] = s / ljj;
+            }
+            if (T > 1) bar.wait();
+        }
+    };
+    if (T == 1) {
+        work(0);
+    } else {
+        std::vector<std::thread> pool;
+        for (int t = 0; t < T; ++t) pool.emplace_back(work, t);
+        for (auto &th : pool) th.join();
+    }
+    if (!ok) return false;
+    for (int64_t j = 0; j < K; ++j) {
+        A[j * K + j] = diag[j];
+        for (int64_t i = j + 1; i < K; ++i) A[j * K + i] = 0.0;
     }
     return true;
 }
@@ -89,7 +147,7 @@ q4_status q4_gptq_hessian(const float *x, int64_t rows, int64_t K, double *H, in
     return Q4_OK;
 }
 
-q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U) {
+q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U, int threads) {
     if (!H || !U || K < 1 || !(damp >= 0.0)) return Q4_ERR_ARG;
     double mean = 0.0;
     for (int64_t i = 0; i < K; ++i) mean += H[i * K + i];
@@ -104,20 +162,30 @@ q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double *U) {
             const double h = 0.5 * (H[i * K + j] + H[j * K + i]);
             A[(K - 1 - i) * K + (K - 1 - j)] = h + (i == j ? damp * mean : 0.0);
         }
-    if (!cholesky_lower(A, K)) return Q4_ERR_ARG;
+    if (!cholesky_lower(A, K, threads)) return Q4_ERR_ARG;
     // column c of L^-1 by forward substitution (x_c = 1 / L[c][c]; x_i for i > c), written
-    // straight into U[K-1-i][K-1-c]
-    std::vector<double> x((size_t)K);
+    // straight into U[K-1-i][K-1-c]; the columns are independent, shared cyclically
     std::fill(U, U + K * K, 0.0);
-    for (int64_t c = 0; c < K; ++c) {
-        x[c] = 1.0 / A[c * K + c];
-        for (int64_t i = c + 1; i < K; ++i) {
-            const double *li = &A[i * K];
-            double s = 0.0;
-            for (int64_t p = c; p < i; ++p) s += li[p] * x[p];
-            x[i] = -s / li[i];
+    const int T = thread_count(threads, K / 64);
+    auto columns = [&](int tid) {
+        std::vector<double> x((size_t)K);
+        for (int64_t c = tid; c < K; c += T) {
+            x[c] = 1.0 / A[c * K + c];
+            for (int64_t i = c + 1; i < K; ++i) {
+                const double *li = &A[i * K];
+                double s = 0.0;
+                for (int64_t p = c; p < i; ++p) s += li[p] * x[p];
+                x[i] = -s / li[i];
+            }
+            for (int64_t i = c; i < K; ++i) U[(K - 1 - i) * K + (K - 1 - c)] = x[i];
         }
-        for (int64_t i = c; i < K; ++i) U[(K - 1 - i) * K + (K - 1 - c)] = x[i];
+    };
+    if (T == 1) {
+        columns(0);
+    } else {
+        std::vector<std::thread> pool;
+        for (int t = 0; t < T; ++t) pool.emplace_back(columns, t);
+        for (auto &th : pool) th.join();
     }
     return Q4_OK;
 }

@@ -37,6 +37,17 @@ def test_prepare_matches_oracle(q4, K):
     assert np.max(np.abs(U - Uo)) <= 1e-9 * np.max(np.abs(Uo))
 
 
+@pytest.mark.parametrize("K", [130, 515])
+def test_prepare_is_the_same_for_any_thread_count(q4, K):
+    X = correlated(2 * K, K, K // 8, K + 1)
+    H = X.astype(np.float64).T @ X.astype(np.float64)
+    U1 = q4.gptq_prepare(H, threads=1)
+    for t in (2, 3, 8):
+        assert np.array_equal(q4.gptq_prepare(H, threads=t), U1)
+    Uo = G.hinv_chol_upper(H)
+    assert np.max(np.abs(U1 - Uo)) <= 1e-9 * np.max(np.abs(Uo))
+
+
 def test_hessian_accumulates_in_fp64(q4):
     X = correlated(300, 48, 5, 1)
     H = q4.gptq_hessian(X[:100], threads=3)
