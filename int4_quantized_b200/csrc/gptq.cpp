@@ -203,27 +203,41 @@ q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U
     const int qmax = qmax_of(bits);
     const int64_t spr = K / group;
     std::vector<int8_t> codes((size_t)(N * K));
+    // rows go through the columns in batches of kRowBatch, so that row k of U is read from
+    // cache by the whole batch; every weight still sees its own updates in k order
+    constexpr int kRowBatch = 8;
     parallel_rows(N, threads, [&](int64_t lo, int64_t hi) {
-        std::vector<double> W((size_t)K);
-        for (int64_t n = lo; n < hi; ++n) {
-            for (int64_t k = 0; k < K; ++k) W[k] = (double)w[n * K + k];
-            float s = 1.0f;
+        std::vector<double> Wb((size_t)(kRowBatch * K));
+        double err[kRowBatch];
+        float s[kRowBatch];
+        for (int64_t n0 = lo; n0 < hi; n0 += kRowBatch) {
+            const int nb = (int)std::min<int64_t>(kRowBatch, hi - n0);
+            for (int r = 0; r < nb; ++r)
+                for (int64_t k = 0; k < K; ++k) Wb[r * K + k] = (double)w[(n0 + r) * K + k];
             for (int64_t k = 0; k < K; ++k) {
-                if (k % group == 0) {
-                    float a = 0.0f;
-                    for (int64_t j = k; j < k + group; ++j) a = std::max(a, std::fabs((float)W[j]));
-                    s = a / (float)qmax;
-                    if (s == 0.0f) s = 1.0f;
-                    scales[n * spr + k / group] = s;
-                }
-                const float t = (float)W[k] / s;
-                float c = std::nearbyint(t);
-                c = std::min(std::max(c, (float)-qmax), (float)qmax);
-                codes[n * K + k] = (int8_t)c;
-                const double wq = (double)(c * s);
-                const double err = (W[k] - wq) / U[k * K + k];
                 const double *uk = U + k * K;
-                for (int64_t j = k + 1; j < K; ++j) W[j] -= err * uk[j];
+                for (int r = 0; r < nb; ++r) {
+                    double *W = &Wb[r * K];
+                    const int64_t n = n0 + r;
+                    if (k % group == 0) {
+                        float a = 0.0f;
+                        for (int64_t j = k; j < k + group; ++j) a = std::max(a, std::fabs((float)W[j]));
+                        s[r] = a / (float)qmax;
+                        if (s[r] == 0.0f) s[r] = 1.0f;
+                        scales[n * spr + k / group] = s[r];
+                    }
+                    const float t = (float)W[k] / s[r];
+                    float c = std::nearbyint(t);
+                    c = std::min(std::max(c, (float)-qmax), (float)qmax);
+                    codes[n * K + k] = (int8_t)c;
+                    const double wq = (double)(c * s[r]);
+                    err[r] = (W[k] - wq) / uk[k];
+                }
+                for (int r = 0; r < nb; ++r) {
+                    double *W = &Wb[r * K];
+                    const double e = err[r];
+                    for (int64_t j = k + 1; j < K; ++j) W[j] -= e * uk[j];
+                }
             }
         }
     });
