@@ -8,8 +8,8 @@ copied until the copies exceed twice the 126 MB L2 (at most 64 copies), and the 
 cycle through them, so that every call reads its weights from HBM. `--reps` calls are
 captured in one CUDA graph (launched `--warmup` times untimed, then `--batches` times
 between CUDA events): the per-call time is the batch time over `--reps`, back-to-back
-device time without the host's launch cost. Printed as one JSON line: the median per-call
-time over the batches and the achieved rates (GB/s of the algorithmic bytes: payload +
+device time without the host's launch cost. Printed as one JSON line: the median and the
+90th percentile of the per-call time over the batches and the achieved rates (at the median) (GB/s of the algorithmic bytes: payload +
 scales for qgemm, fp32 input + payload + scales for qpack; TFLOP/s for qgemm).
 `--static` declares the weights static (Q4_QGEMM_WEIGHTS_STATIC), so each call may
 stream its weights while the one before it ends.
@@ -100,7 +100,9 @@ def main() -> int:
     torch.cuda.synchronize()
     del graph
     us = statistics.median(times)
+    p90 = sorted(times)[min(len(times) - 1, int(round(0.9 * (len(times) - 1))))]
     out = {"kind": a.kind, "N": a.N, "K": a.K, "bits": a.bits, "group": a.group, "us_median": round(us, 3),
+           "us_p90": round(p90, 3),
            "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1), "copies": ncopy, "calls_per_graph": a.reps}
     if a.kind == "qgemm":
         out.update(M=a.M, x="bf16" if a.bf16 else "f32", static=a.static,
