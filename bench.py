@@ -1,29 +1,30 @@
 #!/usr/bin/env python
-"""Benchmark of the grouped-RTN int4/int8 hot path on B200 (one JSON line on stdout).
+"""Benchmark of the grouped-RTN int4/int8 quantized GEMV on B200 (one JSON line on stdout).
 
-One step = one pass of the whole hot path over one batch of the 4096x4096 workload
-(W ~ N(0, 0.02) with 0.1 % 20x outliers, int4 g=128 and int8 g=128, x ~ N(0, 1) at
-M = 1 and M = 8):
-  qpack(W, int4, 128), qgemm(x1), qgemm(x8)  then  qpack(W, int8, 128), qgemm(x1), qgemm(x8).
-Inputs stay resident in HBM. To keep every kernel reading from HBM rather than L2, the
-step rotates over R = 4 copies of W and R payload slots per format, and each GEMV reads
-the slot written two steps earlier (more than the 126 MB L2 is touched in between).
-Each of the R rotation phases is one CUDA graph; step i replays graph i % R.
+Headline (the decode GEMV of the pages' "La vitesse" section, at its largest single-GPU
+configuration): one step = one decode token through a Llama-7B-shaped linear stack,
+32 layers x {q, k, v, o: 4096x4096; gate, up: 11008x4096; down: 4096x11008} = 224
+quantized GEMVs at M = 1, int4 with one fp32 scale per 128 weights, 3,440,377,856 bytes
+of packed weights + scales. The step has data flow (each layer reads what the one before
+wrote) and runs as one launch of the persistent decode-stack kernel (q4_stack_run). The
+weights (3.4 GB) are far beyond the 126 MB L2, so every step streams them from HBM.
 
-value    = algorithmic HBM bytes of all kernels of a step (qpack: 4 B/weight read +
-           payload + scales written; GEMV: payload + scales + x read, y written) x steps
-           x ranks / max-over-ranks device time, in GB/s.
-roofline = the kernel with the largest share of step time, timed with CUDA events over
-           graphs that replay only that kernel (same buffers, same rotation).
-e2e      = the same step through the public API from pinned host buffers, with the H2D
-           copy of W and x and the D2H copy of every y inside the timed region.
-prefill  = the M = 2048 bf16 prefill qgemm (K = 4096, N = 14336) in TFLOP/s.
-decode_stack = the 224 GEMVs of a Llama-7B-shaped stack per token step, one CUDA graph per
-           step, at M = 1, 4, 16 (int4 g128 and int8 per channel): us per step and GB/s.
-cpu_baseline = the oracle (single-threaded C) on a bounded sample of the same step.
+value    = packed weights + scales per step x steps x ranks / max-over-ranks device time,
+           in GB/s (x and y, 0.3 MB per step, are not counted).
+roofline = the step's one kernel: achieved = bytes per launch / mean launch time (CUDA
+           events on the launching stream) against the measured HBM copy bandwidth.
+e2e      = the same step through the public API with the token's activations copied from
+           pinned host memory and the last layer's output copied back, every step.
+Sections: decode_stack (the same step as CUDA graphs of qgemm calls, and int8 with one
+scale per output channel), gemv (single qgemm calls on the 4096x4096 and 1024x1024
+matrices), mlp70b (the 70B-shaped MLP matrices at int4 g64), prefill (M = 2048 bf16 GEMM,
+TFLOP/s), qpack (quantize + pack of the 4096x4096 matrix), cpu_baseline (the oracle on a
+bounded sample of the step).
 
---impl reference times the oracle alone on that sample (there is no reference
-implementation to install: the source pages hold no code for a GPU).
+--impl reference times the oracle alone on that sample (the source pages hold no GPU code
+to install as a reference).
+--case ... times one library call on a seeded shape (see `bench.py --case -h`); profiles
+point a profiler at these command lines.
 """
 from __future__ import annotations
 
@@ -46,9 +47,9 @@ import numpy as np  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "W4/W8 quantized GEMV HBM GB/s (% of peak); prefill qGEMM TFLOP/s"
-WORKLOAD = "mid"          # 4096x4096 with outliers, int4 g128 + int8 g128, M in {1, 8}
-ROT = 4                   # rotating copies of W / payload slots (4 x 67 MB > L2)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+STACK_KERNEL = "gemv_stack_int4_g128_llama7b_M1"
 
 
 # ----------------------------------------------------------------------------------------
@@ -84,19 +85,6 @@ def max_over_ranks(ms: float, device=None) -> float:
 def job_throughput(bytes_per_step: int, steps: int, world: int, ms: float) -> float:
     """Whole-job GB/s: every rank moves bytes_per_step per step (weak scaling) in ms."""
     return bytes_per_step * steps * world / (ms / 1e3) / 1e9
-
-
-def step_bytes(N, K, formats, Ms):
-    """Algorithmic bytes per kernel of one step: {key: bytes}."""
-    out = {}
-    n = N * K
-    for bits, g in formats:
-        pay = n * bits // 8
-        sc = 4 * n // g
-        out[f"qpack_int{bits}_g{g}"] = 4 * n + pay + sc
-        for M in Ms:
-            out[f"gemv_int{bits}_g{g}_M{M}"] = pay + sc + 4 * M * K + 4 * M * N
-    return out
 
 
 # ----------------------------------------------------------------------------------------
@@ -187,78 +175,103 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------------------
-def oracle_sample(N, K, formats, Ms, budget_s=10.0, rows=256):
-    """Time the oracle on a bounded sample of the step: `rows` rows of W, all formats.
+def stack_step_bytes(bits=4, group=128) -> int:
+    """Packed weights + scales of the Llama-7B-shaped step (config arithmetic, no GPU)."""
+    n = sum(N * K for _, N, K in (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                                     ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)))
+    n *= 32
+    if group is None:
+        scales = 32 * (4 * 4096 + 2 * 11008 + 4096) * 4
+    else:
+        scales = n // group * 4
+    return n * bits // 8 + scales
 
-    Returns (GB/s in the same algorithmic-byte accounting, seconds used, description)."""
+
+def oracle_sample(budget_s=10.0, rows=192):
+    """The oracle's quantized matmul on a bounded sample of the decode step: `rows` rows of
+    the first layer's q (K = 4096) and down (K = 11008) matrices, packed by the oracle from
+    the seeded recipe, x from seeds 4 / 5. Returns (GB/s of payload + scales, seconds,
+    description)."""
     import oracle
 
-    wl = workloads.WORKLOADS[WORKLOAD]
-    w = workloads.weight(wl.matrices[0])[:rows].copy()
-    xs = {M: workloads.activations(M, K, wl.x_seed(K)) for M in Ms}
-    per_pass = sum(step_bytes(rows, K, formats, Ms).values())
+    wl = workloads.WORKLOADS["llama7b"]
+    mats = [wl.matrices[0], wl.matrices[6]]
+    jobs = []
+    for m in mats:
+        w = workloads.weight(m)[:rows].copy()
+        payload, scales, _ = oracle.pack(w, 4, 128)
+        x = workloads.activations(1, m.K, wl.x_seed(m.K))
+        jobs.append((x, payload, scales, rows, m.K, payload.nbytes + scales.nbytes))
+    per_pass = sum(j[5] for j in jobs)
     t0 = time.perf_counter()
     passes = 0
     while True:
-        for bits, g in formats:
-            payload, scales, _ = oracle.pack(w, bits, g)
-            for M in Ms:
-                oracle.qgemm(xs[M], payload, scales, rows, K, bits, g)
+        for x, p, s, n, k, _ in jobs:
+            oracle.qgemm(x, p, s, n, k, 4, 128)
         passes += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
     gbs = per_pass * passes / el / 1e9
-    return gbs, el, f"oracle pack+dequant+fp64 matmul of {rows} of the {N} rows, all formats and M, {passes} passes"
+    return gbs, el, (f"oracle dequant + fp64 matmul (single-threaded C) of {rows} rows of L0.q (K=4096) and "
+                     f"L0.down (K=11008), int4 g128, M=1, {passes} passes")
 
 
-def host_cores_used():
-    return 1  # the oracle is single-threaded C
+def host_info():
+    cpu = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    cpu = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cores_used": 1, "host_cpus": os.cpu_count(), "cpu_model": cpu}
 
 
-# ----------------------------------------------------------------------------------------
+def config_block():
+    return {"workload": "Llama-7B-shaped decode step: 32 layers x {q,k,v,o 4096x4096; gate,up 11008x4096; "
+                        "down 4096x11008} = 224 GEMVs, int4 g128, M=1 (one token), layer data flow",
+            "bytes_per_step": stack_step_bytes(),
+            "weights": "W ~ N(0, 0.02) drawn on the device (torch Philox, seed 100+7*layer+index), packed by qpack",
+            "l2": "3.44 GB of weights per step, >> 126 MB L2: inputs larger than L2",
+            "kernel": "one launch of the persistent decode-stack kernel per step",
+            "parallelism": "replicas (one independent decode stack per GPU)"}
+
+
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return 0
-    wl = workloads.WORKLOADS[WORKLOAD]
-    m = wl.matrices[0]
-    formats = [(b, m.K if g is None else g) for b, g in wl.formats]
     budget = max(2.0, min(20.0, 0.5 * (args.steps + args.warmup)))
-    gbs, el, desc = oracle_sample(m.N, m.K, formats, wl.Ms, budget_s=budget)
-    step_b = sum(step_bytes(m.N, m.K, formats, wl.Ms).values())
+    gbs, el, desc = oracle_sample(budget_s=budget)
+    step_b = stack_step_bytes()
+    hi = host_info()
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_b / (gbs * 1e9) * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_block(),
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": host_cores_used(), "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": hi["cores_used"], "kind": "oracle",
+                         "sample": desc, "host_cpus": hi["host_cpus"], "cpu_model": hi["cpu_model"]},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_block():
-    wl = workloads.WORKLOADS[WORKLOAD]
-    return {"workload": "4096x4096 W~N(0,0.02)+0.1% 20x outliers; qpack int4 g128 + int8 g128; GEMV M=1 and M=8",
-            "N": 4096, "K": 4096, "formats": ["int4 g128", "int8 g128"], "M": list(wl.Ms),
-            "l2": f"inputs rotate over {ROT} copies (>126 MB L2); each GEMV reads payload written 2 steps earlier",
-            "gemv_weights": "static during the step (packed 2 steps earlier): GEMVs are launched with "
-                            "Q4_QGEMM_WEIGHTS_STATIC and stream them while the previous kernel ends",
-            "parallelism": "replicas (one independent problem per GPU)"}
-
-
 # ----------------------------------------------------------------------------------------
-# the sources each bench kernel is built from (the traffic figures are dropped when any changes)
-KERNEL_SOURCES = {"qpack": ("qpack.cu", "common.cuh", "kernels.h"), "gemv": ("gemv.cu", "common.cuh", "kernels.h")}
+# the sources each measured kernel is built from (its ncu traffic figure is dropped when any changes)
+KERNEL_SOURCES = {
+    STACK_KERNEL: ("stack.cu", "gemv_math.cuh", "common.cuh", "kernels.h"),
+}
 
 
 def kernel_source_sha(kernel_key):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int4_quantized_b200", "csrc")
-    for fn in KERNEL_SOURCES[kernel_key.split("_")[0]]:
+    for fn in KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(d, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -282,7 +295,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    import int4_quantized_b200 as q4
+    from int4_quantized_b200 import decode_stack as ds
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -291,72 +304,12 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     peaks, peak_kind = load_peaks()
 
-    wl = workloads.WORKLOADS[WORKLOAD]
-    m = wl.matrices[0]
-    N, K = m.N, m.K
-    formats = [(b, K if g is None else g) for b, g in wl.formats]
-    Ms = list(wl.Ms)
-    w_host = workloads.weight(m)
-    x_host = {M: workloads.activations(M, K, wl.x_seed(K)) for M in Ms}
-
-    W = [torch.from_numpy(w_host).to(dev) for _ in range(ROT)]
-    X = {M: torch.from_numpy(x_host[M]).to(dev) for M in Ms}
-    P = {f: [torch.empty(q4.payload_bytes(N, K, f[0]), dtype=torch.uint8, device=dev) for _ in range(ROT)]
-         for f in formats}
-    S = {f: [torch.empty(q4.num_scales(N, K, f[1]), dtype=torch.float32, device=dev) for _ in range(ROT)]
-         for f in formats}
-    Y = {(f, M): torch.empty((M, N), dtype=torch.float32, device=dev) for f in formats for M in Ms}
-    WS = {(f, M): torch.empty(max(256, q4.qgemm_workspace_bytes(M, N, K, f[0], f[1])), dtype=torch.uint8,
-                              device=dev) for f in formats for M in Ms}
-    for f in formats:
-        for r in range(ROT):
-            q4.qpack(W[r], f[0], f[1], payload=P[f][r], scales=S[f][r])
-    torch.cuda.synchronize()
-
-    def call(kind, f, M, i):
-        wi, gj = i % ROT, (i + ROT // 2) % ROT
-        if kind == "qpack":
-            q4.qpack(W[wi], f[0], f[1], payload=P[f][wi], scales=S[f][wi])
-        else:
-            # the payload read here was packed two steps earlier: static while this step runs
-            q4.qgemm(X[M], P[f][gj], S[f][gj], N, K, f[0], f[1], out=Y[(f, M)], workspace=WS[(f, M)],
-                     weights_static=True)
-
-    plan = []
-    for f in formats:
-        plan.append(("qpack", f, None))
-        for M in Ms:
-            plan.append(("gemv", f, M))
-
-    def key(kind, f, M):
-        return f"qpack_int{f[0]}_g{f[1]}" if kind == "qpack" else f"gemv_int{f[0]}_g{f[1]}_M{M}"
-
-    # qpack: one kernel; qgemm: the stream kernel, plus gemv_prep when it needs a workspace
-    launches_per_step = sum(1 if k == "qpack" else (2 if q4.qgemm_workspace_bytes(M, N, K, f[0], f[1]) else 1)
-                            for k, f, M in plan)
-    kbytes = step_bytes(N, K, formats, Ms)
-    bytes_per_step = sum(kbytes.values())
-
+    stack = ds.build_stack(4, 128, 32, dev)
+    dstack, acts = ds.make_decode_stack(stack, 4)
+    bytes_per_step = ds.stack_bytes(stack)
+    assert bytes_per_step == stack_step_bytes()
     stream = torch.cuda.Stream(device=dev)
-    graphs = []
-    with torch.cuda.stream(stream):
-        for i in range(ROT):  # warm the code paths once outside capture
-            for kind, f, M in plan:
-                call(kind, f, M, i)
-    torch.cuda.synchronize()
-    for i in range(ROT):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for kind, f, M in plan:
-                call(kind, f, M, i)
-        graphs.append(g)
-    per_kernel_graphs = {}
-    for kind, f, M in plan:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(ROT):
-                call(kind, f, M, i)
-        per_kernel_graphs[key(kind, f, M)] = g
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
     def barrier():
@@ -365,8 +318,8 @@ def run_ours(args):
 
     def timed(n_steps):
         with torch.cuda.stream(stream):
-            for i in range(args.warmup):
-                graphs[i % ROT].replay()
+            for _ in range(args.warmup):
+                dstack.run(status)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
@@ -376,165 +329,192 @@ def run_ours(args):
         with sampler:
             with torch.cuda.stream(stream):
                 e0.record(stream)
-                for i in range(n_steps):
-                    graphs[i % ROT].replay()
+                for _ in range(n_steps):
+                    dstack.run(status)
                 e1.record(stream)
             torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1)
-        return ms, sampler.summary()
+        return e0.elapsed_time(e1), sampler.summary()
 
     ms, clocks = timed(args.steps)
     if ClockSampler.rejected(clocks):
         ms, clocks = timed(args.steps)  # measured once more, as the rules ask
         clocks["remeasured"] = True
+    if int(status.item()) != 0:
+        raise RuntimeError(f"decode-stack status word {int(status.item()):#x}: a bounded wait gave up")
+    ms_rank = ms
     ms = max_over_ranks(ms, dev)
     value = job_throughput(bytes_per_step, args.steps, world, ms)
-
-    # per-kernel device time: graphs of ROT launches of one kernel kind, same buffers
-    per_kernel = {}
-    reps = max(1, args.steps // ROT)
-    for k, g in per_kernel_graphs.items():
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                g.replay()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                g.replay()
-            b.record(stream)
-        torch.cuda.synchronize()
-        us = a.elapsed_time(b) * 1e3 / (reps * ROT)
-        per_kernel[k] = {"us": round(us, 3), "bytes": kbytes[k],
-                         "GB/s": round(kbytes[k] / (us * 1e-6) / 1e9, 1),
-                         "frac_hbm": round(kbytes[k] / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
-    dom = max(per_kernel, key=lambda k: per_kernel[k]["us"])
-    d = per_kernel[dom]
-    traffic = ncu_traffic(dom)
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": d["GB/s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": d["frac_hbm"], "traffic": traffic, "peak_kind": peak_kind,
-                "frac_of_8TBs_spec": round(d["GB/s"] / 8000.0, 4)}
-    gemv_best = {k: v for k, v in per_kernel.items() if k.startswith("gemv_int4")}
+    launch_us = ms_rank * 1e3 / args.steps
+    achieved = bytes_per_step / (launch_us * 1e-6) / 1e9
+    roofline = {"kernel": STACK_KERNEL, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": ncu_traffic(STACK_KERNEL),
+                "peak_kind": peak_kind, "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+                "algorithmic_bytes_per_launch": bytes_per_step, "launch_us": round(launch_us, 2)}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": config_block(), "roofline": roofline, "kernels": per_kernel,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        "config": config_block(), "roofline": roofline, "gpu_launches": args.steps, "clocks": clocks,
         "gpu": torch.cuda.get_device_name(dev),
     }
-    if gemv_best:
-        out["gemv_int4_g128"] = gemv_best
-
     if rank == 0 and not args.no_e2e:
-        out["e2e"] = e2e(args, q4, dev, w_host, x_host, N, K, formats, Ms, bytes_per_step, world)
-    if rank == 0 and not args.no_prefill:
-        out["prefill"] = prefill(args, q4, dev, peaks, peak_kind)
-    if rank == 0 and not args.no_mlp70b:
+        out["e2e"] = e2e(args, dstack, acts, bytes_per_step, dev)
+    if rank == 0 and not args.no_sections:
+        out["decode_stack"] = decode_stack_section(args, stack, dev, peaks)
+        del stack, dstack, acts
+        torch.cuda.empty_cache()
+        out["gemv"] = gemv_section(args, dev, peaks)
         out["mlp70b"] = mlp70b_section(args, dev, peaks)
-    if rank == 0 and not args.no_stack:
-        out["decode_stack"] = decode_stack_section(args, dev)
+        out["prefill"] = prefill_section(args, dev, peaks, peak_kind)
+        out["qpack"] = qpack_section(args, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, el, desc = oracle_sample(N, K, formats, Ms, budget_s=args.cpu_seconds)
-        out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": host_cores_used(),
-                               "kind": "oracle", "sample": desc, "seconds": round(el, 2)}
+        gbs, el, desc = oracle_sample(budget_s=args.cpu_seconds)
+        hi = host_info()
+        out["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": hi["cores_used"], "kind": "oracle",
+                               "sample": desc, "seconds": round(el, 2), "host_cpus": hi["host_cpus"],
+                               "cpu_model": hi["cpu_model"]}
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del graphs, per_kernel_graphs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
 
 
-def e2e(args, q4, dev, w_host, x_host, N, K, formats, Ms, bytes_per_step, world):
-    """The step through the public API from pinned host memory, copies included."""
+def e2e(args, dstack, acts, bytes_per_step, dev):
+    """The step through the public API: the token's activations from pinned host memory
+    into the stack's input, one q4_stack_run, the last layer's output back to pinned host
+    memory, every step."""
     import torch
 
-    wp = torch.from_numpy(w_host).pin_memory()
-    xp = {M: torch.from_numpy(x_host[M]).pin_memory() for M in Ms}
-    yp = {(f, M): torch.empty((M, N), dtype=torch.float32).pin_memory() for f in formats for M in Ms}
-    wd = torch.empty_like(wp, device=dev)
-    xd = {M: torch.empty_like(xp[M], device=dev) for M in Ms}
-    h2d = wp.numel() * 4 + sum(x.numel() * 4 for x in xp.values())
-    d2h = sum(y.numel() * 4 for y in yp.values())
+    h_host = acts.h0.cpu().pin_memory()
+    y_last = acts.y[(acts.layers - 1, "down")]
+    y_host = torch.empty_like(y_last, device="cpu").pin_memory()
+    stream = torch.cuda.Stream(device=dev)
 
     def one():
-        wd.copy_(wp, non_blocking=True)
-        for M in Ms:
-            xd[M].copy_(xp[M], non_blocking=True)
-        for f in formats:
-            payload, scales = q4.qpack(wd, f[0], f[1])
-            for M in Ms:
-                y = q4.qgemm(xd[M], payload, scales, N, K, f[0], f[1])
-                yp[(f, M)].copy_(y, non_blocking=True)
+        acts.h0.copy_(h_host, non_blocking=True)
+        dstack.run()
+        y_host.copy_(y_last, non_blocking=True)
 
-    for _ in range(3):
-        one()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 50))
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(n):
-        one()
-    b.record()
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(n):
+            one()
+        b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
     return {"value": round(bytes_per_step / (ms / 1e3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+            "h2d_bytes_per_step": h_host.numel() * 4, "d2h_bytes_per_step": y_host.numel() * 4, "steps": n}
 
 
-def prefill(args, q4, dev, peaks, peak_kind):
-    """M = 2048 bf16 prefill qgemm on the 14336x4096 workload, TFLOP/s per format."""
+def decode_stack_section(args, stack, dev, peaks):
+    """The same decode step run other ways (M = 1 unless said), and int8 per channel."""
+    from int4_quantized_b200 import decode_stack as ds
+
+    def frac(r):
+        r["frac_hbm"] = round(r["GB/s"] / peaks["hbm_gbs"], 4)
+        return r
+
+    reps = 20
+    out = {"workload": "the headline's step; graph modes are CUDA graphs of qgemm calls with weights declared "
+                       "static; M > 1 reads fixed activations",
+           "int4_g128": [frac(ds.time_persistent(stack, 4, reps, fused=True)),
+                         frac(ds.time_graph(stack, 4, 1, reps)),
+                         frac(ds.time_graph(stack, 4, 1, reps, fused=False)),
+                         frac(ds.time_graph(stack, 4, 4, reps)),
+                         frac(ds.time_graph(stack, 4, 16, reps))]}
+    s8 = ds.build_stack(8, None, 32, dev)
+    out["int8_per_channel"] = [frac(ds.time_persistent(s8, 8, reps)), frac(ds.time_graph(s8, 8, 1, reps))]
+    del s8
+    return out
+
+
+def _l2_copies(nbytes):
+    return max(1, min(64, -(-2 * L2_BYTES // nbytes)))
+
+
+def time_calls(call, ncopy, reps=None, warmup=3, batches=5):
+    """Median per-call device time (us) of `call(i)` captured back to back in a CUDA graph
+    (the calls cycle through `ncopy` input copies so the weights come from HBM)."""
     import torch
 
-    wl = workloads.WORKLOADS["prefill"]
-    m = wl.matrices[0]
-    M = wl.Ms[0]
-    N, K = m.N, m.K
-    w = torch.from_numpy(workloads.weight(m)).to(dev)
-    x = workloads.activations_bf16(M, K, wl.x_seed(K)).to(dev)
+    reps = reps or max(10, 2 * ncopy)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            call(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(reps):
+            call(i)
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+        for _ in range(batches):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3 / reps)
+    torch.cuda.synchronize()
+    del graph
+    return statistics.median(times), sorted(times)[-1]
+
+
+def gemv_section(args, dev, peaks):
+    """Single qgemm calls: the 4096x4096 matrix with 20x outliers (int4/int8 g128, M = 1 and 8,
+    inputs rotated beyond L2) and the 1024x1024 matrix (L2-resident; us only)."""
+    import torch
+
+    import int4_quantized_b200 as q4
+
     res = {}
-    for bits, g in wl.formats:
-        g = K if g is None else g
-        payload, scales = q4.qpack(w, bits, g)
-        y = torch.empty((M, N), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(256, q4.qgemm_workspace_bytes(M, N, K, bits, g, torch.bfloat16)), dtype=torch.uint8,
-                         device=dev)
-        for _ in range(3):
-            q4.qgemm(x, payload, scales, N, K, bits, g, out=y, workspace=ws)
-        torch.cuda.synchronize()
-        reps = 10
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            q4.qgemm(x, payload, scales, N, K, bits, g, out=y, workspace=ws)
-        b.record()
-        torch.cuda.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
-        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
-        res[f"int{bits}_g{g}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 2),
-                                  "frac_bf16": round(tf / peaks["bf16_tflops"], 4)}
-    del w
-    return {"workload": "M=2048 K=4096 N=14336, x bf16 (L2-resident inputs, tensor-bound)", "peak_kind": peak_kind,
-            "peak_bf16_tflops": peaks["bf16_tflops"], **res}
+    for wname, fmts, Ms in (("mid", ((4, 128), (8, 128)), (1, 8)), ("small", ((8, 1024), (4, 32)), (1,))):
+        wl = workloads.WORKLOADS[wname]
+        m = wl.matrices[0]
+        w = torch.from_numpy(workloads.weight(m)).to(dev)
+        for bits, g in fmts:
+            p, s = q4.qpack(w, bits, g)
+            nbytes = p.numel() + 4 * s.numel()
+            ncopy = _l2_copies(nbytes) if wname == "mid" else 1
+            P = [p] + [p.clone() for _ in range(ncopy - 1)]
+            S = [s] + [s.clone() for _ in range(ncopy - 1)]
+            for M in Ms:
+                x = torch.from_numpy(workloads.activations(M, m.K, wl.x_seed(m.K))).to(dev)
+                y = torch.empty(M, m.N, device=dev)
+                ws = torch.empty(max(256, q4.qgemm_workspace_bytes(M, m.N, m.K, bits, g)), dtype=torch.uint8,
+                                 device=dev)
+                for static in (False, True):
+                    def call(i):
+                        q4.qgemm(x, P[i % ncopy], S[i % ncopy], m.N, m.K, bits, g, out=y, workspace=ws,
+                                 weights_static=static)
+                    us, us_max = time_calls(call, ncopy)
+                    gbs = nbytes / (us * 1e-6) / 1e9
+                    res[f"{wname}_int{bits}_g{g}_M{M}{'_static' if static else ''}"] = {
+                        "N": m.N, "K": m.K, "us": round(us, 3), "us_max": round(us_max, 3), "GB/s": round(gbs, 1),
+                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4) if wname == "mid" else None,
+                        "l2": "rotated beyond L2" if wname == "mid" else "L2-resident"}
+            del P, S
+    return res
 
 
 def mlp70b_section(args, dev, peaks):
-    """The 70B-shaped MLP matrices (gate/up 28672x8192, down 8192x28672, int4 g64, M = 1).
-
-    Each matrix is packed once on the GPU. Two CUDA graphs of back-to-back calls: rounds of
-    (gate, up), which share a shape, and rounds of (gate, up, down); every call reads
-    another 132 MB matrix than the call before it, and a round (264 or 396 MB) is past the
-    126 MB L2, so the weights come from HBM. The first graph gives the 28672x8192 time per
-    call, the second the time of the three; the 8192x28672 time is their difference
-    (marked "derived"). Both launch modes are timed: plain stream order, and weights
-    declared static.
-    """
+    """The 70B-shaped MLP matrices (gate/up 28672x8192, down 8192x28672, int4 g64, M = 1), each
+    132 MB packed: CUDA graphs of back-to-back calls cycling gate, up, down (396 MB per round,
+    past L2), plain and with weights declared static."""
     import torch
 
     import int4_quantized_b200 as q4
@@ -548,70 +528,152 @@ def mlp70b_section(args, dev, peaks):
         del w
         x = torch.from_numpy(workloads.activations(1, m.K, wl.x_seed(m.K))).to(dev)
         y = torch.empty((1, m.N), dtype=torch.float32, device=dev)
-        mats.append((m, payload, scales, x, y, payload.numel() + 4 * scales.numel()))
-    torch.cuda.synchronize()
-    stream = torch.cuda.Stream(device=dev)
-    nb = mats[0][5]
-    rounds = 10
-
-    def graph_time(seq, static):
-        def run():
-            for _ in range(rounds):
-                for m, p, sc, x, y, _ in seq:
-                    q4.qgemm(x, p, sc, m.N, m.K, bits, group, out=y, weights_static=static)
-        with torch.cuda.stream(stream):
-            run()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            run()
-        ts = []
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                g.replay()
-            for _ in range(5):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                g.replay()
-                b.record(stream)
-                b.synchronize()
-                ts.append(a.elapsed_time(b) * 1e3 / rounds)
-        del g
-        return sorted(ts)[len(ts) // 2]
-
-    def entry(us, nbytes, **kw):
-        gbs = nbytes / (us * 1e-6) / 1e9
-        return {**kw, "us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-
-    out = {"workload": wl.description, "bytes_per_matrix": nb, "calls_per_graph": {"gate_up": 2 * rounds,
-                                                                                  "all3": 3 * rounds}}
+        mats.append((m, payload, scales, x, y))
+    nb = mats[0][1].numel() + 4 * mats[0][2].numel()
+    out = {"workload": wl.description, "bytes_per_matrix": nb}
     for static in (False, True):
-        t_gu = graph_time(mats[:2], static) / 2
-        t_all = graph_time(mats, static)
-        out["int4_g64_static" if static else "int4_g64"] = {
-            "gate_up_28672x8192": entry(t_gu, nb, N=28672, K=8192),
-            "down_8192x28672": entry(t_all - 2 * t_gu, nb, N=8192, K=28672, derived=True),
-            "all3": entry(t_all, 3 * nb),
-        }
+        def call(i):
+            m, p, s, x, y = mats[i % 3]
+            q4.qgemm(x, p, s, m.N, m.K, bits, group, out=y, weights_static=static)
+        us, us_max = time_calls(call, 3, reps=30)
+        gbs = nb / (us * 1e-6) / 1e9
+        out["int4_g64_static" if static else "int4_g64"] = {"us_per_matrix": round(us, 2), "GB/s": round(gbs, 1),
+                                                            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
     return out
 
 
-def decode_stack_section(args, dev):
-    """The 224-GEMV Llama-7B-shaped stack, one CUDA graph per token step (M = 1, 4, 16)."""
-    from int4_quantized_b200 import decode_stack as ds
+def prefill_section(args, dev, peaks, peak_kind):
+    """M = 2048 bf16 prefill qgemm on the 14336x4096 workload, TFLOP/s per format."""
+    import torch
 
-    out = {"workload": "Llama-7B-shaped linear stack: 32 x (4 x 4096x4096, 2 x 11008x4096, 4096x11008), "
-                       "W ~ N(0, 0.02) drawn on the device, weights read from HBM every step",
-           "gemvs_per_step": 7 * 32}
-    for bits, group, key in ((4, 128, "int4_g128"), (8, None, "int8_per_channel")):
-        stack = ds.build_stack(bits, group, 32, dev)
-        out[key] = [ds.time_stack(stack, bits, M, reps=10, weights_static=True) for M in (1, 4, 16)]
-        out[key + "_plain"] = [ds.time_stack(stack, bits, M, reps=10, weights_static=False) for M in (1, 4, 16)]
-        del stack
-    return out
+    import int4_quantized_b200 as q4
+
+    wl = workloads.WORKLOADS["prefill"]
+    m = wl.matrices[0]
+    M = wl.Ms[0]
+    N, K = m.N, m.K
+    w = torch.from_numpy(workloads.weight(m)).to(dev)
+    x = workloads.activations_bf16(M, K, wl.x_seed(K)).to(dev)
+    res = {}
+    for bits, g in wl.formats:
+        g = K if g is None else g
+        payload, scales = q4.qpack(w, bits, g)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+
+        def call(i):
+            q4.qgemm(x, payload, scales, N, K, bits, g, out=y)
+        us, us_max = time_calls(call, 1, reps=10)
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        res[f"int{bits}_g{g}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 2),
+                                  "frac_bf16": round(tf / peaks["bf16_tflops"], 4)}
+    del w
+    return {"workload": "M=2048 K=4096 N=14336, x bf16 (tensor-bound)", "peak_kind": peak_kind,
+            "peak_bf16_tflops": peaks["bf16_tflops"], **res}
+
+
+def qpack_section(args, dev, peaks):
+    """qpack of the 4096x4096 matrix (fp32 in, payload + scales out), inputs rotated beyond L2."""
+    import torch
+
+    import int4_quantized_b200 as q4
+
+    wl = workloads.WORKLOADS["mid"]
+    m = wl.matrices[0]
+    w0 = torch.from_numpy(workloads.weight(m)).to(dev)
+    res = {}
+    for bits, g in ((4, 128), (8, 128)):
+        p0, s0 = q4.qpack(w0, bits, g)
+        nbytes = 4 * w0.numel() + p0.numel() + 4 * s0.numel()
+        ncopy = _l2_copies(nbytes)
+        W = [w0] + [w0.clone() for _ in range(ncopy - 1)]
+        P = [p0] + [p0.clone() for _ in range(ncopy - 1)]
+        S = [s0] + [s0.clone() for _ in range(ncopy - 1)]
+
+        def call(i):
+            q4.qpack(W[i % ncopy], bits, g, payload=P[i % ncopy], scales=S[i % ncopy])
+        us, us_max = time_calls(call, ncopy)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[f"int{bits}_g{g}"] = {"us": round(us, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del W, P, S
+    return {"workload": "4096x4096 W~N(0,0.02)+0.1% 20x outliers; bytes = 4 B/weight read + payload + scales",
+            **res}
+
+
+# ----------------------------------------------------------------------------------------
+def run_case(argv):
+    """One library call on a seeded shape, timed; the command line profilers are pointed at."""
+    ap = argparse.ArgumentParser(prog="bench.py --case", description=(
+        "qgemm N K bits group [M] | qpack N K bits group | stack bits group. W ~ N(0, 0.02) and x ~ N(0, 1) "
+        "from a fixed device seed; inputs copied until they exceed twice the L2 (at most 64 copies); --reps "
+        "calls captured in one CUDA graph and timed with CUDA events. The stack case is the Llama-7B-shaped "
+        "decode step (group 0 = one scale per output channel)."))
+    ap.add_argument("kind", choices=["qgemm", "qpack", "stack"])
+    ap.add_argument("shape", type=int, nargs="+")
+    ap.add_argument("--bf16", action="store_true", help="x in bfloat16 (qgemm)")
+    ap.add_argument("--static", action="store_true", help="weights declared static (qgemm)")
+    ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--batches", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=32, help="stack: decoder layers")
+    a = ap.parse_args(argv)
+    import torch
+
+    import int4_quantized_b200 as q4
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gen = torch.Generator(device=dev).manual_seed(0)
+    if a.kind == "stack":
+        from int4_quantized_b200 import decode_stack as ds
+
+        bits, group = a.shape[0], (a.shape[1] if len(a.shape) > 1 else 128)
+        stack = ds.build_stack(bits, group or None, a.layers, dev)
+        r = ds.time_persistent(stack, bits, a.reps, a.warmup)
+        print(json.dumps({"kind": "stack", "bits": bits, "group": group or "per-channel", "layers": a.layers, **r}),
+              flush=True)
+        return 0
+    N, K, bits, group = a.shape[:4]
+    M = a.shape[4] if len(a.shape) > 4 else 1
+    w = torch.randn(N, K, device=dev, generator=gen) * 0.02
+    payload, scales = q4.qpack(w, bits, group)
+    pbytes = payload.numel() + 4 * scales.numel()
+    if a.kind == "qgemm":
+        del w
+        x = torch.randn(M, K, device=dev, generator=gen)
+        if a.bf16:
+            x = x.to(torch.bfloat16)
+        y = torch.empty(M, N, device=dev)
+        ncopy = _l2_copies(pbytes)
+        P = [payload] + [payload.clone() for _ in range(ncopy - 1)]
+        S = [scales] + [scales.clone() for _ in range(ncopy - 1)]
+        ws = torch.empty(max(256, q4.qgemm_workspace_bytes(M, N, K, bits, group, x.dtype)), dtype=torch.uint8,
+                         device=dev)
+
+        def call(i):
+            q4.qgemm(x, P[i % ncopy], S[i % ncopy], N, K, bits, group, out=y, workspace=ws, weights_static=a.static)
+        nbytes = pbytes
+    else:
+        ncopy = _l2_copies(4 * w.numel() + pbytes)
+        W = [w] + [w.clone() for _ in range(ncopy - 1)]
+        P = [payload] + [payload.clone() for _ in range(ncopy - 1)]
+        S = [scales] + [scales.clone() for _ in range(ncopy - 1)]
+
+        def call(i):
+            q4.qpack(W[i % ncopy], bits, group, payload=P[i % ncopy], scales=S[i % ncopy])
+        nbytes = 4 * w.numel() + pbytes
+    us, us_max = time_calls(call, ncopy, a.reps, a.warmup, a.batches)
+    out = {"kind": a.kind, "N": N, "K": K, "bits": bits, "group": group, "us_median": round(us, 3),
+           "us_max": round(us_max, 3), "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1), "copies": ncopy}
+    if a.kind == "qgemm":
+        out.update(M=M, x="bf16" if a.bf16 else "f32", static=a.static,
+                   TFLOPs=round(2.0 * M * N * K / (us * 1e-6) / 1e12, 2))
+    print(json.dumps(out), flush=True)
+    return 0
 
 
 def main():
+    if "--case" in sys.argv:
+        i = sys.argv.index("--case")
+        return run_case(sys.argv[i + 1:])
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -619,10 +681,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sections", action="store_true", help="headline only (no decode_stack/gemv/mlp70b/"
+                                                               "prefill/qpack sections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-stack", action="store_true", help="skip the whole-stack decode section")
-    ap.add_argument("--no-mlp70b", action="store_true", help="skip the 70B-shaped MLP section")
+    ap.add_argument("--case", nargs=argparse.REMAINDER, help="time one library call (see --case -h)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

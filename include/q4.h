@@ -71,6 +71,11 @@ Q4_API int q4_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 Q4_API const char *q4_status_str(q4_status s);
 
+/* The CUDA error behind the last Q4_ERR_CUDA returned to this host thread: the
+ * failing step, cudaGetErrorName and cudaGetErrorString, or "" if none. The string
+ * belongs to the library and stays valid until the next call on this thread. */
+Q4_API const char *q4_last_cuda_error(void);
+
 /* Bytes of packed codes for rows*cols weights: rows*cols*bits/8 (pack()'s
  * payload length check on the "量化推理" page). Returns 0 for invalid
  * arguments (negative sizes, bits not 4/8, odd rows*cols with bits = 4). */
@@ -218,6 +223,87 @@ Q4_API q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t 
 Q4_API q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,
                 const float *scales, int64_t N, int64_t K, int bits, int64_t group, float *y,
                 uint32_t *status_word, void *stream);
+
+/*
+ * ---- Decode stack: every GEMV of a decode step in one persistent kernel ("Huit
+ * bits, puis quatre", section "La vitesse": a step made of many short kernels is
+ * bound by launches and pipeline fills; the weights pay off once the GEMVs are
+ * fused so that they wait on memory). One row of activations per GEMV, the
+ * arithmetic and accuracy of qgemm.
+ *
+ * GEMVs are grouped in levels: the GEMVs of level l may read (as x) what GEMVs of
+ * levels < l write (as y), and nothing that GEMVs of level >= l write. Inside one
+ * launch, level l starts reading x only once every GEMV of level l - 1 has written
+ * all of y; weights stream continuously across levels. A transformer layer is four
+ * levels: q|k|v, o, gate|up, down.
+ */
+typedef struct q4_stack_gemv {
+    const uint8_t *payload;  /* [N][K*bits/8] from qpack of an [N][K] matrix, 16-byte aligned */
+    const float *scales;     /* [N*K/group] from the same qpack */
+    const void *x;           /* [K] activations, fp32 or bf16 (the stack's xt), 16-byte aligned */
+    float *y;                /* [N] output; must not overlap another GEMV's y of the same level */
+    int64_t N, K;
+    int64_t group;           /* divides K, multiple of 32 (group = K: one scale per row) */
+    int32_t level;           /* 0 for the first; each next GEMV has the same level or one more */
+    int32_t reserved;        /* 0 */
+} q4_stack_gemv;
+
+/* Host-side record of a prepared stack (filled by q4_stack_prepare, read by
+ * q4_stack_run; plain bytes, may be copied). */
+typedef struct q4_stack_plan {
+    uint64_t opaque[32];
+} q4_stack_plan;
+
+/* Workspace bytes q4_stack_prepare needs for these GEMVs: the GEMV and level tables
+ * (one 2D TMA descriptor per GEMV), one counter per 128-row block and per level, and
+ * the partial sums of row blocks split between CTAs (296 x 128 floats x 2). Returns 0
+ * for arguments q4_stack_prepare rejects. */
+Q4_API size_t q4_stack_workspace_bytes(const q4_stack_gemv *gemvs, int32_t count, int bits, q4_xdtype xt);
+
+/*
+ * q4_stack_prepare -- validate the GEMVs and write the stack's tables into the
+ * workspace, then synchronize `stream` (this call is not for stream capture).
+ *   gemvs      HOST array of count GEMVs, in level order
+ *   bits       4 or 8, for every GEMV; all GEMVs must map to the same kernel variant
+ *              (the same groups per 128-byte tile: e.g. all group = 128, or all
+ *              one scale per row)
+ *   xt         dtype of every x
+ *   workspace  device memory of q4_stack_workspace_bytes(...) bytes, 256-byte
+ *              aligned, owned by the caller; it belongs to the plan until the
+ *              caller stops running it. The weights, x and y pointers are stored:
+ *              they must stay valid, and payload and scales must not change, while
+ *              the plan is run.
+ *   plan       out
+ * Errors: Q4_ERR_ARG (null pointers, bits, sizes, levels out of order, reserved != 0),
+ * Q4_ERR_UNSUPPORTED (group not a multiple of 32 dividing K, mixed kernel variants,
+ * misaligned payload or x, N or K > 2^30), Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
+ */
+Q4_API q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, q4_xdtype xt,
+                void *workspace, size_t workspace_bytes, q4_stack_plan *plan, void *stream);
+
+/*
+ * q4_stack_run -- one launch of the prepared stack on `stream` (capturable in a CUDA
+ * graph). Every y is written; results are deterministic and, per GEMV, within
+ * qgemm's accuracy bound for the x it read.
+ *   status_word  optional device uint32; Q4_STATUS_TIMEOUT is OR-ed into it if a
+ *              bounded wait gave up (every y is then invalid; the workspace stays
+ *              usable).
+ * Two runs of one plan (or plans sharing a workspace) must not overlap in time.
+ * Errors: Q4_ERR_ARG (not a prepared plan), Q4_ERR_CUDA (e.g. the grid cannot be
+ * resident at once on this device).
+ */
+Q4_API q4_status q4_stack_run(const q4_stack_plan *plan, uint32_t *status_word, void *stream);
+
+/*
+ * q4_stack_set_wait_limit -- the bound of every wait inside the stack kernel, in
+ * nanoseconds (1e9 after q4_stack_prepare). A wait that reaches it gives up: the run
+ * then ends without waiting further, ORs Q4_STATUS_TIMEOUT into the status word, and
+ * leaves the workspace ready for the next run. A bound shorter than the waits of a
+ * working run (microseconds) makes that run give up; a caller that watches for a
+ * broken producer upstream may want a bound shorter than the default.
+ * Errors: Q4_ERR_ARG (not a prepared plan).
+ */
+Q4_API q4_status q4_stack_set_wait_limit(q4_stack_plan *plan, uint64_t nanoseconds);
 
 /*
  * ---- GPTQ host quantizer ("Huit bits, puis quatre", section "Arrondir mieux :

@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "Q4Error", "lib", "lib_path", "payload_bytes", "num_scales", "qgemm_workspace_bytes",
-    "qpack", "qdequant", "qgemm", "qgemm_noalloc", "gptq_hessian", "gptq_prepare", "gptq_quantize", "gptq_pack", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
+    "qpack", "qdequant", "qgemm", "qgemm_noalloc", "StackGemv", "DecodeStack", "gptq_hessian", "gptq_prepare", "gptq_quantize", "gptq_pack", "NOALLOC_SCRATCH_BYTES", "Q4_OK", "Q4_ERR_ARG", "Q4_ERR_UNSUPPORTED", "Q4_ERR_CUDA",
     "Q4_ERR_NONFINITE", "Q4_ERR_WORKSPACE", "Q4_ERR_SCRATCH_LIMIT", "Q4_X_F32", "Q4_X_BF16", "Q4_QGEMM_WEIGHTS_STATIC", "STATUS_NONFINITE", "STATUS_TIMEOUT",
 ]
 
@@ -45,7 +45,10 @@ _lock = threading.Lock()
 class Q4Error(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {lib().q4_status_str(code).decode()} (status {code})")
+        msg = f"{what}: {lib().q4_status_str(code).decode()} (status {code})"
+        if code == Q4_ERR_CUDA:
+            msg += f": {lib().q4_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 def lib() -> ctypes.CDLL:
@@ -62,6 +65,7 @@ def lib() -> ctypes.CDLL:
                 L.q4_version.restype = i32
                 L.q4_status_str.argtypes = [i32]
                 L.q4_status_str.restype = ctypes.c_char_p
+                L.q4_last_cuda_error.restype = ctypes.c_char_p
                 L.q4_payload_bytes.argtypes = [i64, i64, i32]
                 L.q4_payload_bytes.restype = sz
                 L.q4_num_scales.argtypes = [i64, i64, i64]
@@ -79,6 +83,14 @@ def lib() -> ctypes.CDLL:
                 L.qgemm_ex.restype = i32
                 L.qgemm_noalloc.argtypes = [vp, i32, i64, vp, vp, i64, i64, i32, i64, vp, vp, vp]
                 L.qgemm_noalloc.restype = i32
+                L.q4_stack_workspace_bytes.argtypes = [vp, ctypes.c_int32, i32, i32]
+                L.q4_stack_workspace_bytes.restype = sz
+                L.q4_stack_prepare.argtypes = [vp, ctypes.c_int32, i32, i32, vp, sz, vp, vp]
+                L.q4_stack_prepare.restype = i32
+                L.q4_stack_run.argtypes = [vp, vp, vp]
+                L.q4_stack_run.restype = i32
+                L.q4_stack_set_wait_limit.argtypes = [vp, ctypes.c_uint64]
+                L.q4_stack_set_wait_limit.restype = i32
                 L.q4_gptq_hessian.argtypes = [vp, i64, i64, vp, i32]
                 L.q4_gptq_hessian.restype = i32
                 L.q4_gptq_prepare.argtypes = [vp, i64, ctypes.c_double, vp, i32]
@@ -232,6 +244,73 @@ def qgemm_noalloc(x: torch.Tensor, payload: torch.Tensor, scales: torch.Tensor, 
         _check(lib().qgemm_noalloc(_ptr(x), xt, M, _ptr(payload), _ptr(scales), N, K, bits, group,
                                    _ptr(out), _ptr(status), _stream(x.device)), "qgemm_noalloc")
     return out
+
+
+# ---- decode stack: every GEMV of a decode step in one persistent kernel -----------------
+
+class _StackGemvC(ctypes.Structure):
+    _fields_ = [("payload", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("group", ctypes.c_int64),
+                ("level", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class StackGemv:
+    """One GEMV of a decode stack: y[N] = W'[N, K] x[K] (x float32 or bfloat16)."""
+
+    def __init__(self, payload: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor,
+                 N: int, K: int, group: int, level: int):
+        _cuda(payload, "payload", torch.uint8)
+        _cuda(scales, "scales", torch.float32)
+        _cuda(x, "x")
+        _cuda(y, "y", torch.float32)
+        if x.numel() != K or y.numel() != N:
+            raise ValueError("x must hold K values and y N values")
+        self.payload, self.scales, self.x, self.y = payload, scales, x, y
+        self.N, self.K, self.group, self.level = int(N), int(K), int(group), int(level)
+
+
+class DecodeStack:
+    """A prepared stack of GEMVs (q4_stack_prepare); run() is one launch of all of them.
+
+    Levels: the GEMVs of level l may read what GEMVs of earlier levels write; every GEMV
+    of level l - 1 has finished writing before level l reads its x. The workspace and the
+    tensors of every GEMV are held for the life of the object.
+    """
+
+    def __init__(self, gemvs: Sequence[StackGemv], bits: int):
+        if not gemvs:
+            raise ValueError("empty stack")
+        dt = gemvs[0].x.dtype
+        if dt not in (torch.float32, torch.bfloat16) or any(g.x.dtype != dt for g in gemvs):
+            raise TypeError("every x must have the same dtype, float32 or bfloat16")
+        self.gemvs = list(gemvs)
+        self.bits = bits
+        self.device = gemvs[0].payload.device
+        xt = Q4_X_BF16 if dt == torch.bfloat16 else Q4_X_F32
+        arr = (_StackGemvC * len(gemvs))()
+        for i, g in enumerate(gemvs):
+            arr[i] = _StackGemvC(g.payload.data_ptr(), g.scales.data_ptr(), g.x.data_ptr(), g.y.data_ptr(),
+                                 g.N, g.K, g.group, g.level, 0)
+        n = len(gemvs)
+        need = int(lib().q4_stack_workspace_bytes(ctypes.byref(arr), n, bits, xt))
+        if need == 0:
+            raise Q4Error(Q4_ERR_ARG, "stack_workspace_bytes")
+        self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        self._plan = (ctypes.c_uint64 * 32)()
+        with torch.cuda.device(self.device):
+            _check(lib().q4_stack_prepare(ctypes.byref(arr), n, bits, xt, _ptr(self.workspace), need,
+                                          ctypes.byref(self._plan), _stream(self.device)), "stack_prepare")
+        self.weight_bytes = sum(g.payload.numel() + 4 * g.scales.numel() for g in gemvs)
+
+    def set_wait_limit(self, nanoseconds: int) -> None:
+        """Bound of every wait inside the kernel (default 1e9 ns); see q4_stack_set_wait_limit."""
+        _check(lib().q4_stack_set_wait_limit(ctypes.byref(self._plan), int(nanoseconds)), "stack_set_wait_limit")
+
+    def run(self, status: Optional[torch.Tensor] = None) -> None:
+        if status is not None:
+            _cuda(status, "status", torch.int32)
+        with torch.cuda.device(self.device):
+            _check(lib().q4_stack_run(ctypes.byref(self._plan), _ptr(status), _stream(self.device)), "stack_run")
 
 
 # ---- GPTQ host quantizer (host arrays; the computation runs in libq4's C++ code) ----------

@@ -5,11 +5,23 @@
 // that survives a call is qgemm_noalloc's cached scratch address per device.
 #include <cuda_runtime.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "kernels.h"
 
 namespace q4 {
+
+// The last failing CUDA call of this host thread, for q4_last_cuda_error().
+thread_local char g_last_cuda_error[160] = "";
+
+q4_status cuda_error(cudaError_t e, const char *where) {
+    if (e == cudaSuccess) return Q4_OK;
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s (%s)", where, cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return Q4_ERR_CUDA;
+}
+
 // rowscale.cu: out[n] = scales[n / rows_per_scale] for n < N
 cudaError_t launch_expand_row_scales(const float *scales, int64_t rows_per_scale, int64_t N, float *out,
                                      cudaStream_t st);
@@ -47,6 +59,8 @@ q4_status check_format(int64_t rows, int64_t cols, int bits, int64_t group, int6
 
 inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
+inline q4_status cuda_status(cudaError_t e, const char *where) { return q4::cuda_error(e, where); }
+
 // Path selection and workspace layout of one qgemm call.
 struct QgemmPlan {
     q4::GemvPlan gemv;    // the fused GEMV plan (for the row-scale group when rps > 1)
@@ -72,7 +86,7 @@ q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q
         if (N % p->rps != 0) return Q4_ERR_ARG;  // no [N][K] matrix has such groups
         p->group = K;
     }
-    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, p->group, kPlanSMs, &p->gemv))
+    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, p->group, xt == Q4_X_BF16, kPlanSMs, &p->gemv))
         return Q4_ERR_UNSUPPORTED;
     p->prefill = q4::prefill_supported(M, N, K, bits, p->group, xt == Q4_X_BF16);
     p->scale_bytes = p->rps > 1 ? align256((size_t)N * 4) : 0;
@@ -90,12 +104,14 @@ void *g_noalloc_ptr[kMaxDevices] = {};
 
 q4_status noalloc_scratch(void **out) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return Q4_ERR_CUDA;
+    const cudaError_t ge = cudaGetDevice(&dev);
+    if (ge != cudaSuccess) return cuda_status(ge, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return Q4_ERR_CUDA;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress");
         g_noalloc_ptr[dev] = p;
     }
     *out = g_noalloc_ptr[dev];
@@ -106,7 +122,9 @@ q4_status noalloc_scratch(void **out) {
 
 extern "C" {
 
-int q4_version(void) { return 100; }
+int q4_version(void) { return 200; }
+
+const char *q4_last_cuda_error(void) { return q4::g_last_cuda_error; }
 
 const char *q4_status_str(q4_status s) {
     switch (s) {
@@ -143,7 +161,7 @@ q4_status qpack(const float *w, int64_t rows, int64_t cols, int bits, int64_t gr
     if (!w || !payload || !scales) return Q4_ERR_ARG;
     cudaError_t e = q4::launch_qpack(w, n, bits, group, payload, scales, status_word,
                                      as_stream(stream), device_sms());
-    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return cuda_status(e, "qpack launch");
 }
 
 q4_status qdequant(const uint8_t *payload, const float *scales, int64_t rows, int64_t cols,
@@ -155,7 +173,7 @@ q4_status qdequant(const uint8_t *payload, const float *scales, int64_t rows, in
     if (!payload || !scales || !w_out) return Q4_ERR_ARG;
     cudaError_t e = q4::launch_qdequant(payload, scales, n, bits, group, w_out, as_stream(stream),
                                         device_sms());
-    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return cuda_status(e, "qdequant launch");
 }
 
 size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
@@ -184,7 +202,8 @@ q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payloa
     if (p.rps > 1) {
         // one scale per row, written by the kernel just before: no early start
         float *rs = static_cast<float *>(workspace);
-        if (q4::launch_expand_row_scales(scales, p.rps, N, rs, s) != cudaSuccess) return Q4_ERR_CUDA;
+        const cudaError_t re = q4::launch_expand_row_scales(scales, p.rps, N, rs, s);
+        if (re != cudaSuccess) return cuda_status(re, "row-scale launch");
         sc = rs;
         early = false;
     }
@@ -196,7 +215,7 @@ q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payloa
         e = q4::launch_gemv(p.gemv, x, xt == Q4_X_BF16, M, payload, sc, N, K, p.group, y, ws, status_word, early,
                             s);
     }
-    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return cuda_status(e, p.prefill ? "prefill launch" : "gemv launch");
 }
 
 q4_status qgemm(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payload,

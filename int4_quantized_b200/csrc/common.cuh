@@ -129,13 +129,15 @@ Q4_DEVINL uint64_t global_ns() {
     return t;
 }
 // Bounded wait: retries the suspending try_wait; the global timer bounds the whole wait
-// at about one second, so a lost arrival can never hang the GPU. Returns false on timeout.
-Q4_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// at limit_ns (one second by default), so a lost arrival can never hang the GPU. Returns
+// false on timeout.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+Q4_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > 1000000000ull) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 // 2D tiled TMA load global -> shared, completion counted in bytes on `bar`.

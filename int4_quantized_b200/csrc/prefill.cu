@@ -447,22 +447,6 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            p = nullptr;
-        return reinterpret_cast<EncodeTiledFn>(p);
-    }();
-    return fn;
-}
-
 constexpr size_t smem_bytes() {
     return 1024 + (size_t)kStages * kXBytes + (size_t)kAStages * kABytes + (size_t)kStages * kPBytesMax +
            (2 * kStages + 2 * kAStages + 5) * 8 + 16;
