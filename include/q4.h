@@ -208,7 +208,10 @@ Q4_API q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t 
  *            libq4, one per device, created by the CUDA runtime with the
  *            library's module. The first call on each device (with that device
  *            current) looks up its address once and caches it; make that first
- *            call before any stream capture on the device. Nothing in the
+ *            call before any stream capture on the device. The cached address
+ *            lives as long as the device's primary context: after cudaDeviceReset
+ *            (or anything else that destroys it), do not call qgemm_noalloc again
+ *            in the same process. Nothing in the
  *            scratch has to start at zero: each call writes every byte it reads.
  *   Limit:   problems with q4_qgemm_workspace_bytes(...) greater than
  *            Q4_NOALLOC_SCRATCH_BYTES are rejected with Q4_ERR_SCRATCH_LIMIT
@@ -348,7 +351,8 @@ Q4_API q4_status q4_gptq_prepare(const double *H, int64_t K, double damp, double
  *   threads  worker threads over rows (0 = all); the result does not depend on it
  * Cost: N * K^2 / 2 multiply-subtracts. Requirements: bits 4 or 8, group
  * divides K, N * K even for int4.
- * Errors: Q4_ERR_ARG, Q4_ERR_NONFINITE (W holds NaN or Inf; outputs untouched).
+ * Errors: Q4_ERR_ARG, Q4_ERR_NONFINITE (W holds NaN or Inf, or an ill-conditioned U
+ * drove a corrected weight outside the fp32 range; outputs untouched).
  */
 Q4_API q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U, int bits,
                 int64_t group, uint8_t *payload, float *scales, int threads);

@@ -597,13 +597,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-bool encode_payload_map(CUtensorMap *tm, const uint8_t *payload, int64_t N, int64_t K, int bits) {
+bool encode_payload_map(CUtensorMap *tm, const uint8_t *payload, int64_t N, int64_t K, int bits, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const uint64_t rowbytes = (uint64_t)K * bits / 8;
     const cuuint64_t dims[2] = {rowbytes, (cuuint64_t)N};
     const cuuint64_t strides[1] = {rowbytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kTileBytes, (cuuint32_t)kTileRows};
+    const cuuint32_t box[2] = {(cuuint32_t)kTileBytes, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(payload), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -698,7 +698,7 @@ cudaError_t launch_gemv(const GemvPlan &pl, const void *x, bool x_bf16, int64_t 
                         cudaStream_t st) {
     if (!encode_fn()) return cudaErrorNotSupported;
     CUtensorMap tm;
-    if (!encode_payload_map(&tm, payload, N, K, pl.bits)) return cudaErrorInvalidValue;
+    if (!encode_payload_map(&tm, payload, N, K, pl.bits, kRowsPerCta)) return cudaErrorInvalidValue;
     char *w = static_cast<char *>(ws);
     GemvArgs a;
     a.scales = scales;

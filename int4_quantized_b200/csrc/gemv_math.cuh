@@ -123,20 +123,22 @@ Q4_DEVINL void load_x8(const void *x, int64_t idx, float (&v)[8]) {
 }
 
 // ---- decode of the packed codes ------------------------------------------------------
-// bf16x2 a - b and a * 1 + c, rounded to nearest (exact here: small integers).
-Q4_DEVINL uint32_t bsub2(uint32_t a, uint32_t b) {
+// bf16x2 a * b + c, rounded to nearest (exact here: small integers).
+Q4_DEVINL uint32_t bfma2(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
-// int4: nibbles 0..3 and 16..19 of v (u = code + 8) -> the bf16 pair of codes.
+constexpr uint32_t kBf16One2 = 0x3f803f80u;  // (1.0, 1.0)
+// int4: nibbles 0..3 and 16..19 of v (u = code + 8) -> the bf16 pair of codes:
+// (128 + u) * 1 - 136.
 Q4_DEVINL uint32_t codes4(uint32_t v) {
-    return bsub2(and_or(v, 0x000f000fu, 0x43004300u), 0x43084308u);  // (128 + u) - 136
+    return bfma2(and_or(v, 0x000f000fu, 0x43004300u), kBf16One2, 0xc308c308u);
 }
-// int8: bytes 0 and 2 of v (two's complement codes) -> the bf16 pair of codes.
+// int8: bytes 0 and 2 of v (two's complement codes) -> the bf16 pair of codes:
+// (128 + (c & 127)) * 1 - (128, or 256 when c < 0).
 Q4_DEVINL uint32_t codes8(uint32_t v) {
-    // (128 + (c & 127)) - (128, or 256 when c < 0)
-    return bsub2(and_or(v, 0x007f007fu, 0x43004300u), and_or(v, 0x00800080u, 0x43004300u));
+    return bfma2(and_or(v, 0x007f007fu, 0x43004300u), kBf16One2, and_or(v, 0x00800080u, 0xc300c300u));
 }
 
 // A fragment of MMA j of a segment from one lane's words of row g (w0) and row g+8 (w1).
@@ -280,6 +282,290 @@ Q4_DEVINL void stage_fixed(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
     }
 }
 
+
+
+// ======================================================================================
+// One row of x: a per-stage choice between exact integer digits and exact bf16 pieces
+// ======================================================================================
+// When the activations of a 128-byte stage span a dynamic range of at most 2^21 (every
+// nonzero |x| >= 2^(E - 21), where max |x| < 2^E), each one is written as the 40-bit
+// fixed-point integer X = rint(x * 2^(38 - E)), split into five balanced base-256 digits
+// (one int8 MMA column each), and the codes enter the tensor core as int8 (int8 codes as
+// stored; int4 nibbles as 16 * code). Every product and every sum of a scale group is then
+// an exact integer; the only rounding of x is X's, at most 2^(E - 39) = 2^-18 of the
+// element's own magnitude. Stages with a wider range (or extreme exponents) use the bf16
+// pieces instead (exact products for any finite x). Both are integrated per lane into two
+// fp32 sums (rows g and g + 8 of the warp's tile).
+//
+// Slot of one stage: the B fragments (either format: the same size) and a header.
+//   pieces: k16 MMAs x 16 lanes stored x 8 bytes, columns (hi, mid, lo, 0) [P = 3] or
+//           (x, 0, 0, 0) [P = 1]
+//   digits: k32 MMAs x 32 lanes x 8 bytes, column c holds digit 4 - c, columns 5-7 zero
+//   header: int mode (1 = digits), float f = 2^(E - 38) (x 2^-4 for int4, whose A operand
+//           is 16 * code)
+template <int BITS>
+__host__ __device__ constexpr int slot1_data() { return BITS == 4 ? 2048 : 1024; }
+template <int BITS>
+__host__ __device__ constexpr int slot1_bytes() { return slot1_data<BITS>() + 16; }
+
+Q4_DEVINL float pow2i(int e) { return __int_as_float((e + 127) << 23); }  // 2^e, e in [-126, 127]
+
+// Smallest E with max|x| < 2^E from the bits of max|x| (> 0, finite).
+Q4_DEVINL int exp_above(uint32_t mx) {
+    const int be = (int)(mx >> 23);
+    if (be > 0) return be - 126;
+    return (32 - __clz((int)mx)) - 149;  // subnormal: mx * 2^-149 with mx < 2^23
+}
+
+// Decision for a stage from the bits of its max |x| and of its smallest nonzero |x|
+// (0x7f800000 when every x is 0): digits when the range condition holds and E leaves the
+// scale factors normal; *E_out is E (0 for an all-zero stage).
+Q4_DEVINL bool digits_ok(uint32_t mx, uint32_t mn, int *E_out) {
+    if (mx >= 0x7f800000u) return false;  // Inf or NaN: the pieces carry them
+    if (mx == 0) {
+        *E_out = 0;
+        return true;
+    }
+    const int E = exp_above(mx);
+    *E_out = E;
+    if (E < -60 || E > 100) return false;
+    const int te = E - 21;  // threshold 2^te
+    const uint32_t thr = te >= -126 ? (uint32_t)(te + 127) << 23 : (te >= -149 ? 1u << (te + 149) : 0u);
+    return mn >= thr;
+}
+
+// Balanced base-256 digits of X = rint(x * 2^(38 - E)), |X| < 2^38: returns the 64-bit
+// word whose bytes 0..4 are the digits (two's complement int8), digit p of weight 256^p.
+Q4_DEVINL uint64_t digits5(float x, int E) {
+    const int sh = 38 - E;  // 38 - E in [-62, 98]: two exact power-of-two steps
+    const int s1 = sh > 64 ? 64 : sh;
+    const float v = (x * pow2i(s1)) * pow2i(sh - s1);
+    const long long X = __float2ll_rn(v);
+    return ((uint64_t)X + 0x8080808080ull) ^ 0x8080808080ull;
+}
+
+// out[p] = byte p of (a, b, c, d), in that order.
+Q4_DEVINL void bytes_transpose4(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t (&out)[4]) {
+    const uint32_t t0 = prmt(a, b, 0x5140u), t1 = prmt(a, b, 0x7362u);
+    const uint32_t t2 = prmt(c, d, 0x5140u), t3 = prmt(c, d, 0x7362u);
+    out[0] = prmt(t0, t2, 0x5410u);
+    out[1] = prmt(t0, t2, 0x7632u);
+    out[2] = prmt(t1, t3, 0x5410u);
+    out[3] = prmt(t1, t3, 0x7632u);
+}
+// Byte 0 of each of a, b, c, d, in that order.
+Q4_DEVINL uint32_t bytes0(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return prmt(prmt(a, b, 0x0040u), prmt(c, d, 0x0040u), 0x5410u);
+}
+
+// Digit-format B fragments of 8 consecutive k (offset kk in the stage, a multiple of 8):
+// one lane slice of one k32 MMA. int4: b0 = the even k of the word, b1 = the odd k (the
+// low and high nibbles of its bytes); int8: b0 = k 0..3, b1 = k 4..7.
+template <int BITS, int L>
+Q4_DEVINL void digits_unit(uint2 *slot, int kk, const float (&v)[8], int E) {
+    constexpr int KTID = BITS == 4 ? L / 4 : L / 8;  // k32 MMAs per segment
+    const int byte = BITS == 4 ? (kk >> 1) : kk;
+    const int sl = byte / (4 * L), t = (byte % (4 * L)) / L;
+    const int j = BITS == 4 ? (byte % L) / 4 : (byte % L) / 8;
+    const int i = sl * KTID + j;
+    uint64_t D[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) D[q] = digits5(v[q], E);
+    const int q0[4] = {BITS == 4 ? 0 : 0, BITS == 4 ? 2 : 1, BITS == 4 ? 4 : 2, BITS == 4 ? 6 : 3};
+    const int o = BITS == 4 ? 1 : 4;  // b1 takes the values q0[] + o
+    uint32_t T0[4], T1[4];
+    bytes_transpose4((uint32_t)D[q0[0]], (uint32_t)D[q0[1]], (uint32_t)D[q0[2]], (uint32_t)D[q0[3]], T0);
+    bytes_transpose4((uint32_t)D[q0[0] + o], (uint32_t)D[q0[1] + o], (uint32_t)D[q0[2] + o], (uint32_t)D[q0[3] + o],
+                     T1);
+    const uint32_t h0 = bytes0((uint32_t)(D[q0[0]] >> 32), (uint32_t)(D[q0[1]] >> 32), (uint32_t)(D[q0[2]] >> 32),
+                               (uint32_t)(D[q0[3]] >> 32));
+    const uint32_t h1 = bytes0((uint32_t)(D[q0[0] + o] >> 32), (uint32_t)(D[q0[1] + o] >> 32),
+                               (uint32_t)(D[q0[2] + o] >> 32), (uint32_t)(D[q0[3] + o] >> 32));
+    auto at = [&](int col) -> uint2 & { return slot[frag_idx(i, 0, 4 * col + t, 1, 32, true)]; };
+    at(0) = make_uint2(h0, h1);  // digit 4
+#pragma unroll
+    for (int p = 3; p >= 0; --p) at(4 - p) = make_uint2(T0[p], T1[p]);
+#pragma unroll
+    for (int col = 5; col < 8; ++col) at(col) = make_uint2(0u, 0u);
+}
+
+// Piece-format B fragments of 8 consecutive k, every stored column written (the columns
+// no piece uses are zero).
+template <int BITS, int L>
+Q4_DEVINL void pieces_unit(uint2 *slot, int kk, const float (&v)[8], int P) {
+    frag_unit<BITS, L>(slot, kk, 0, v, P, 4, 1, 16, true);
+    float z[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) z[q] = 0.f;
+    for (int vm = 1; vm * P < 4; ++vm) frag_unit<BITS, L>(slot, kk, vm, z, P, 4, 1, 16, true);
+}
+
+// A fragment of k32 int8 MMA j of a segment (digits format) from one lane's words of row
+// g (w0) and row g + 8 (w1). int4: byte (u_hi << 4 | u_lo), u = code + 8: (u << 4) ^ 0x80
+// is the int8 16 * code.
+template <int BITS, int L>
+Q4_DEVINL void unpack_a8(uint32_t (&a)[4], const uint32_t (&w0)[L / 4], const uint32_t (&w1)[L / 4], int j) {
+    if constexpr (BITS == 4) {
+        const uint32_t x0 = w0[j], x1 = w1[j];
+        a[0] = ((x0 << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // even k of row g
+        a[1] = ((x1 << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // even k of row g + 8
+        a[2] = (x0 & 0xF0F0F0F0u) ^ 0x80808080u;         // odd k of row g
+        a[3] = (x1 & 0xF0F0F0F0u) ^ 0x80808080u;         // odd k of row g + 8
+    } else {
+        a[0] = w0[2 * j];
+        a[1] = w1[2 * j];
+        a[2] = w0[2 * j + 1];
+        a[3] = w1[2 * j + 1];
+    }
+}
+
+// One stage of one row of x in the pieces format: the group sums of the two piece columns
+// this lane holds, scaled by the group's fp32 scale, go into y0 (row g) and y1 (row g + 8).
+template <int BITS, int L, int GPS, bool FULL>
+Q4_DEVINL void stage1_pieces(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
+                             const uint32_t (&A1)[kTileBytes / (4 * L)][L / 4], const uint8_t *slot, int lane,
+                             const float *s0p, const float *s1p, int nsl, float &y0, float &y1) {
+    constexpr int SPS = kTileBytes / (4 * L);
+    constexpr int KTI = BITS == 4 ? L / 2 : L / 4;
+    constexpr int KTS = SPS * KTI;
+    constexpr int NG = GPS > 0 ? GPS : 1;
+    constexpr int IPG = KTS / NG;
+    constexpr int CH = NG < 4 ? NG : 4;
+    const uint8_t *frl = slot + (lane & 15) * 16;
+    // lanes 16-31 read the fragments of lanes 0-15: their columns (4-7) repeat columns
+    // 0-3 and must not be counted
+    const bool own = (lane & 2) == 0;
+    float c[CH][4];
+    uint4 bq[1];
+    auto flush = [&](int q, float (&cc)[4]) {
+        if (own) {
+            y0 = fmaf(s0p[q], cc[0] + cc[1], y0);
+            y1 = fmaf(s1p[q], cc[2] + cc[3], y1);
+        }
+    };
+    auto valid = [&](int q) { return q < NG && (FULL || q * (SPS / NG) < nsl); };
+#pragma unroll
+    for (int i = 0; i < KTS; ++i) {
+        const int sl = i / KTI, j = i % KTI, q = i / IPG, ch = q % CH;
+        if (FULL || sl < nsl) {
+            if (CH > 1 && i % IPG == 0 && q >= CH) flush(q - CH, c[ch]);
+            uint32_t af[4];
+            unpack_a<BITS, L>(af, A0[sl], A1[sl], j);
+            uint32_t b0, b1;
+            load_b<1, 16, true>(frl, i, 0, bq, b0, b1);
+            if (i % IPG == 0)
+                mma_bf16_z(c[ch], af, b0, b1);
+            else
+                mma_bf16(c[ch], af, b0, b1);
+            if constexpr (CH == 1) {
+                const bool last = GPS > 0 ? (i % IPG == IPG - 1)
+                                          : (FULL ? i == KTS - 1 : (j == KTI - 1 && sl == nsl - 1));
+                if (last) flush(q, c[0]);
+            }
+        }
+    }
+    if constexpr (CH > 1) {
+#pragma unroll
+        for (int q = 0; q < NG; ++q)
+            if (valid(q) && !valid(q + CH)) flush(q, c[q % CH]);
+    }
+}
+
+// The same stage in the digits format: exact int32 group sums; a lane's column pair
+// (digits d, d - 1) combines exactly as 256 * c0 + c1 and is scaled by the group's scale
+// times fl (2^(E - 38), the lane's pair weight 256^(3 - 2t) and the int4 factor 2^-4).
+template <int BITS, int L, int GPS, bool FULL>
+Q4_DEVINL void stage1_digits(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
+                             const uint32_t (&A1)[kTileBytes / (4 * L)][L / 4], const uint8_t *slot, int lane,
+                             const float *s0p, const float *s1p, int nsl, float fl, float &y0, float &y1) {
+    constexpr int SPS = kTileBytes / (4 * L);
+    constexpr int KTI = BITS == 4 ? L / 4 : L / 8;  // k32 MMAs per segment
+    constexpr int KTS = SPS * KTI;
+    constexpr int NG = GPS > 0 ? GPS : 1;
+    constexpr int IPG = KTS / NG;
+    constexpr int CH = NG < 4 ? NG : 4;
+    const uint8_t *frl = slot + lane * 16;
+    int c[CH][4];
+    uint4 bq[1];
+    auto flush = [&](int q, int (&cc)[4]) {
+        const int p0 = cc[0] * 256 + cc[1], p1 = cc[2] * 256 + cc[3];
+        y0 = fmaf(s0p[q] * fl, __int2float_rn(p0), y0);
+        y1 = fmaf(s1p[q] * fl, __int2float_rn(p1), y1);
+    };
+    auto valid = [&](int q) { return q < NG && (FULL || q * (SPS / NG) < nsl); };
+#pragma unroll
+    for (int i = 0; i < KTS; ++i) {
+        const int sl = i / KTI, j = i % KTI, q = i / IPG, ch = q % CH;
+        if (FULL || sl < nsl) {
+            if (CH > 1 && i % IPG == 0 && q >= CH) flush(q - CH, c[ch]);
+            uint32_t af[4];
+            unpack_a8<BITS, L>(af, A0[sl], A1[sl], j);
+            uint32_t b0, b1;
+            load_b<1, 32, true>(frl, i, 0, bq, b0, b1);
+            if (i % IPG == 0)
+                mma_s8_16832_z(c[ch], af, b0, b1);
+            else
+                mma_s8_16832(c[ch], af, b0, b1);
+            if constexpr (CH == 1) {
+                const bool last = GPS > 0 ? (i % IPG == IPG - 1)
+                                          : (FULL ? i == KTS - 1 : (j == KTI - 1 && sl == nsl - 1));
+                if (last) flush(q, c[0]);
+            }
+        }
+    }
+    if constexpr (CH > 1) {
+#pragma unroll
+        for (int q = 0; q < NG; ++q)
+            if (valid(q) && !valid(q + CH)) flush(q, c[q % CH]);
+    }
+}
+
+// Builds the slot of one stage from its activations x[k0, k0 + STAGEK) (zeros past K): the
+// calling warp's lanes take 8 k each (all 32 for int4, 16 for int8), decide the format
+// together and write every byte of the slot (header by lane 0).
+template <int BITS, int L, bool XBF16, bool CG>
+Q4_DEVINL void build_slot1(uint8_t *slot, const void *x, int k0, int K, int P, int lane) {
+    constexpr int STAGEK = kTileBytes * 8 / BITS;
+    constexpr int LANES = STAGEK / 8;
+    const int kk = 8 * lane;
+    float v[8];
+    if (lane < LANES && k0 + kk < K) {
+        load_x8<XBF16, CG>(x, k0 + kk, v);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = 0.f;
+    }
+    uint32_t mx = 0, mn = 0x7f800000u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t a = __float_as_uint(v[q]) & 0x7fffffffu;
+        mx = max(mx, a);
+        if (a != 0) mn = min(mn, a);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    int E = 0;
+    const bool dig = digits_ok(mx, mn, &E);
+    uint2 *s2 = reinterpret_cast<uint2 *>(slot);
+    if (lane < LANES) {
+        if (dig)
+            digits_unit<BITS, L>(s2, kk, v, E);
+        else
+            pieces_unit<BITS, L>(s2, kk, v, P);
+    }
+    if (lane == 0) {
+        int *h = reinterpret_cast<int *>(slot + slot1_data<BITS>());
+        h[0] = dig ? 1 : 0;
+        h[1] = E;
+    }
+}
+
+// The lane's multiplier of the digits format: 2^(E - 38) times its column pair's weight
+// 256^(3 - 2t) (t = lane & 3; pairs (4, 3), (2, 1), (0, -)), times 2^-4 for int4.
+template <int BITS>
+Q4_DEVINL float digit_lane_factor(int E, int t) {
+    return pow2i(E - 38 + 24 - 16 * t - (BITS == 4 ? 4 : 0));
+}
 
 }  // namespace gm
 }  // namespace q4

@@ -11,6 +11,7 @@
 // Each output row only ever reads its own weights, so rows run on separate threads; the
 // operations on every weight are those of the definition, in its order.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <condition_variable>
 #include <cstdint>
@@ -203,6 +204,10 @@ q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U
     const int qmax = qmax_of(bits);
     const int64_t spr = K / group;
     std::vector<int8_t> codes((size_t)(N * K));
+    // scales are kept here until the whole walk is known to be finite: an ill-conditioned U
+    // can push a corrected weight past the fp32 range, and then nothing is written
+    std::vector<float> sc((size_t)(N * spr));
+    std::atomic<bool> nonfinite{false};
     // rows go through the columns in batches of kRowBatch, so that row k of U is read from
     // cache by the whole batch; every weight still sees its own updates in k order
     constexpr int kRowBatch = 8;
@@ -221,10 +226,16 @@ q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U
                     const int64_t n = n0 + r;
                     if (k % group == 0) {
                         float a = 0.0f;
-                        for (int64_t j = k; j < k + group; ++j) a = std::max(a, std::fabs((float)W[j]));
+                        bool ok = true;
+                        for (int64_t j = k; j < k + group; ++j) {
+                            const float v = (float)W[j];
+                            ok = ok && std::isfinite(v);
+                            a = std::max(a, std::fabs(v));
+                        }
+                        if (!ok) nonfinite.store(true, std::memory_order_relaxed);
                         s[r] = a / (float)qmax;
                         if (s[r] == 0.0f) s[r] = 1.0f;
-                        scales[n * spr + k / group] = s[r];
+                        sc[n * spr + k / group] = s[r];
                     }
                     const float t = (float)W[k] / s[r];
                     float c = std::nearbyint(t);
@@ -241,6 +252,8 @@ q4_status q4_gptq_quantize(const float *w, int64_t N, int64_t K, const double *U
             }
         }
     });
+    if (nonfinite.load()) return Q4_ERR_NONFINITE;
+    std::memcpy(scales, sc.data(), sc.size() * sizeof(float));
     const int64_t n = N * K;
     if (bits == 8) {
         std::memcpy(payload, codes.data(), (size_t)n);

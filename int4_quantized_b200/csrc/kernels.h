@@ -60,8 +60,8 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_fn();
-// The GEMV's map of an [N][K*bits/8] payload: tiles of 128 rows x 128 bytes, 128B swizzle.
-bool encode_payload_map(CUtensorMap *tm, const uint8_t *payload, int64_t N, int64_t K, int bits);
+// The GEMV's map of an [N][K*bits/8] payload: tiles of box_rows rows x 128 bytes, 128B swizzle.
+bool encode_payload_map(CUtensorMap *tm, const uint8_t *payload, int64_t N, int64_t K, int bits, int box_rows);
 
 // ---- prefill GEMM (tcgen05) ----------------------------------------------------------
 // bf16 x with M >= 64, K and group multiples of 64: the tensor-memory GEMM of prefill.cu.

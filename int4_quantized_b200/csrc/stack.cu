@@ -43,12 +43,18 @@ namespace {
 
 using namespace gm;
 
-constexpr int kConsumers = 8;
+// One CTA per SM: fifteen consumer warps (16 weight rows each) on 240-row tiles and one
+// producer warp. Registers: 512 threads x 128 fill the SM's 64K; shared memory stays near
+// 160 KB so that about 70 KB of the SM's 228 KB remain L1, which holds the lines of scales
+// the consumers read (a 128-byte line serves a row over many consecutive stages).
+constexpr int kConsumers = 15;
 constexpr int kConsumerThreads = 32 * kConsumers;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kRing = 5;                   // payload stages in flight per CTA
-constexpr int kSmemBudget = 115200;        // two CTAs per SM
-constexpr int kCtasPerSm = 2;
+constexpr int kSRows = 16 * kConsumers;            // 240 weight rows per tile
+constexpr int kSTile = kTileBytes * kSRows;        // 30 KB of codes per tile
+constexpr int kRing = 4;                           // tiles in flight per CTA
+constexpr int kSmemBudget = 163840;
+constexpr int kCtasPerSm = 1;
 
 struct alignas(64) StackEntry {
     CUtensorMap tm;        // 2D map of the payload: {row bytes, N}, box 128 x 128, 128B swizzle
@@ -75,11 +81,12 @@ struct StackLevel {
 struct StackArgs {
     const StackEntry *ent;
     const StackLevel *lev;
-    int *task_cnt;         // [n_tasks] arrivals of the CTAs sharing a row block
-    int *level_done;       // [L] completed row blocks per level
+    int *task_cnt;         // [n_tasks][15] arrivals of the CTAs sharing a row block, per warp
+    int *level_done;       // [L] completed (row block, warp) pairs per level
     int *finished;         // CTAs done with the launch
     int *tflag;            // set when a wait gave up: the last CTA also resets task_cnt
-    float *partial;        // [G][2][128] partial sums
+    float *partial;        // [G][2][240] partial sums
+    const int *ustart;     // [L][G + 1] first tile of each CTA's range in each level
     uint32_t *status;
     int G, L, n_tasks;
     int P;                 // pieces per activation: 3 (fp32 x) or 1 (bf16 x)
@@ -108,11 +115,6 @@ Q4_DEVINL void tma_load_2d_g(void *dst, const CUtensorMap *tmap, uint64_t *bar, 
         : "memory");
 }
 
-// Tiles [u0, u1) of a level with U tiles that CTA c of G owns.
-Q4_DEVINL void cta_range(int64_t U, int c, int G, int64_t &u0, int64_t &u1) {
-    u0 = U * c / G;
-    u1 = U * (c + 1) / G;
-}
 // The CTA that owns tile u of a level with U tiles.
 Q4_DEVINL int cta_of(int64_t u, int64_t U, int G) { return (int)(((u + 1) * G - 1) / U); }
 
@@ -120,6 +122,29 @@ Q4_DEVINL int cta_of(int64_t u, int64_t U, int G) { return (int)(((u + 1) * G - 
 Q4_DEVINL int locate(const StackEntry *ent, int e, int e_end, int64_t u) {
     while (e + 1 < e_end && u >= ent[e + 1].unit_base) ++e;
     return e;
+}
+
+// Position of a tile: GEMV e, row block rb, k-stage s.
+struct Cursor {
+    int e, rb, s;
+};
+Q4_DEVINL Cursor cursor_at(const StackEntry *ent, const StackLevel &lv, int64_t u) {
+    Cursor cu;
+    cu.e = locate(ent, lv.e0, lv.e0 + lv.ne, u);
+    const int ul = (int)(u - ent[cu.e].unit_base);  // < R * S < 2^31
+    const int S = ent[cu.e].S;
+    cu.rb = ul / S;
+    cu.s = ul - cu.rb * S;
+    return cu;
+}
+// One tile forward; true when it moved to another GEMV (whose fields must be reloaded).
+Q4_DEVINL bool cursor_next(Cursor &cu, int S, int R) {
+    if (++cu.s < S) return false;
+    cu.s = 0;
+    if (++cu.rb < R) return false;
+    cu.rb = 0;
+    ++cu.e;
+    return true;
 }
 
 Q4_DEVINL bool wait_counter(const int *p, int target, uint64_t limit_ns) {
@@ -133,32 +158,30 @@ Q4_DEVINL bool wait_counter(const int *p, int target, uint64_t limit_ns) {
 }
 
 template <int BITS, int L, int GPS, bool XBF16>
-__global__ void __maxnreg__(96) gemv_stack(const StackArgs a) {
+__global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     constexpr int SPS = kTileBytes / (4 * L);
     constexpr int KTI = BITS == 4 ? L / 2 : L / 4;
     constexpr int KTS = SPS * KTI;
     constexpr int WPT = L / 4;
     constexpr int STAGEK = kTileBytes * 8 / BITS;
     constexpr int GS = GPS > 0 ? GPS : 1;
-    constexpr int FSLOT = KTS * 16 * 8;  // piece bytes of one tile (16 lanes stored)
+    constexpr int FSLOT = slot1_bytes<BITS>();  // B fragments of one tile + format header
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *ring = smem;                                                  // kRing x 16 KB
-    float *scl = reinterpret_cast<float *>(ring + kRing * kTileWords);    // kRing x [128][GS]
-    float *redc = scl + kRing * kTileRows * GS;                           // [128][8]
-    uint8_t *bbuf = reinterpret_cast<uint8_t *>(redc + kTileRows * 8);     // ucap x FSLOT
+    uint8_t *ring = smem;                                                  // kRing x 30 KB
+    uint8_t *bbuf = ring + kRing * kSTile;                             // ucap x FSLOT
     uint64_t *full = reinterpret_cast<uint64_t *>(bbuf + (size_t)a.ucap * FSLOT);
     uint64_t *empty = full + kRing;
-    int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: last arriver, [1]: timed out
+    int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: a wait of this CTA gave up
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, G = a.G;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRing; ++i) {
-            mbar_init(full + i, 1 + 32);  // the TMA's expect_tx arrival + 32 lanes' scale copies
+            mbar_init(full + i, 1);  // the TMA's expect_tx arrival
             mbar_init(empty + i, kConsumers);
         }
-        flag[0] = flag[1] = 0;
+        flag[0] = 0;
         fence_barrier_init();
     }
     __syncthreads();
@@ -172,34 +195,26 @@ __global__ void __maxnreg__(96) gemv_stack(const StackArgs a) {
         for (int i = 0; i < kRing; ++i) issued[i] = 0;
         for (int l = 0; l < a.L; ++l) {
             const StackLevel lv = a.lev[l];
-            int64_t u0, u1;
-            cta_range(lv.U, c, G, u0, u1);
-            int e = lv.e0;
-            int e_acq = -1;
-            for (int64_t u = u0; u < u1; ++u) {
-                e = locate(a.ent, e, lv.e0 + lv.ne, u);
-                const StackEntry &E = a.ent[e];
-                if (e != e_acq) {
-                    tmap_acquire(&E.tm);
-                    e_acq = e;
+            const int *us = a.ustart + (size_t)l * (G + 1);
+            const int64_t u0 = us[c];
+            const int n = us[c + 1] - us[c];
+            if (n == 0) continue;
+            Cursor cu = cursor_at(a.ent, lv, u0);
+            const StackEntry *E = a.ent + cu.e;
+            int S = E->S, R = E->R;
+            tmap_acquire(&E->tm);
+            for (int i = 0; i < n; ++i) {
+                if (i > 0 && cursor_next(cu, S, R)) {
+                    E = a.ent + cu.e;
+                    S = E->S;
+                    R = E->R;
+                    tmap_acquire(&E->tm);
                 }
-                const int64_t ul = u - E.unit_base;
-                const int rb = (int)(ul / E.S), s = (int)(ul - (int64_t)rb * E.S);
                 if (round > 0 && !timed_out) timed_out = !mbar_wait(empty + slot, (uint32_t)((round - 1) & 1), a.wait_ns);
                 if (lane == 0 && !timed_out) {
-                    mbar_arrive_expect_tx(full + slot, kTileWords);
-                    tma_load_2d_g(ring + slot * kTileWords, &E.tm, full + slot, s * kTileBytes, rb * kTileRows);
+                    mbar_arrive_expect_tx(full + slot, kSTile);
+                    tma_load_2d_g(ring + slot * kSTile, &E->tm, full + slot, cu.s * kTileBytes, cu.rb * kSRows);
                 }
-                // the tile's scales: GS per row (the groups of the stage), clamped to the row
-                const int gbase = GPS > 0 ? s * GPS : (s * STAGEK) / E.group;
-                const int ng = min(GS, E.spr - gbase);
-                float *dst = scl + slot * kTileRows * GS;
-                for (int r = lane; r < kTileRows; r += 32) {
-                    const int n = min(rb * kTileRows + r, E.N - 1);
-                    const float *src = E.scales + (size_t)n * E.spr + gbase;
-                    for (int q = 0; q < ng; ++q) cp_async4(dst + r * GS + q, src + q);
-                }
-                cp_async_arrive(full + slot);
                 ++issued[slot];
                 if (++slot == kRing) { slot = 0; ++round; }
             }
@@ -219,157 +234,185 @@ __global__ void __maxnreg__(96) gemv_stack(const StackArgs a) {
             const int off = sl * 4 * L + t * L;
             aoff[sl] = pr * kTileBytes + (((off >> 4) ^ (pr & 7)) << 4) + (off & 15);
         }
-        const int fl = lane & 15;
-        float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
+        float ys0 = 0.f, ys1 = 0.f;  // this lane's share of rows pr and pr + 8
         int slot = 0, round = 0;
         for (int l = 0; l < a.L; ++l) {
             const StackLevel lv = a.lev[l];
-            int64_t u0, u1;
-            cta_range(lv.U, c, G, u0, u1);
-            if (u0 == u1) continue;
+            const int *us = a.ustart + (size_t)l * (G + 1);
+            const int64_t u0 = us[c];
+            const int n = us[c + 1] - us[c];
+            if (n == 0) continue;
             if (l > 0) {
-                // the activations of this level are complete once every row block of the
-                // previous level is
+                // the activations of this level are complete once every warp of every row
+                // block of the previous level has published its rows
                 if (ct == 0 && !timed_out) {
-                    timed_out = !wait_counter(a.level_done + (l - 1), a.lev[l - 1].T, a.wait_ns);
+                    timed_out = !wait_counter(a.level_done + (l - 1), kConsumers * a.lev[l - 1].T, a.wait_ns);
                     __threadfence();
                 }
                 named_barrier_sync(1, kConsumerThreads);
             }
-            int e = locate(a.ent, lv.e0, lv.e0 + lv.ne, u0);
-            int64_t chunk_end = u0;
-            for (int64_t u = u0; u < u1; ++u) {
-                if (u == chunk_end) {
-                    // pieces of x for the next ucap tiles (every warp is done with the last ones)
-                    if (u != u0) named_barrier_sync(1, kConsumerThreads);
-                    chunk_end = min(u1, u + a.ucap);
-                    constexpr int IPT = STAGEK / 8;  // 8-k items per tile
-                    const int items = (int)(chunk_end - u) * IPT;
-                    int ei = e;
-                    for (int it = ct; it < items; it += kConsumerThreads) {
-                        const int j = it / IPT, kk = 8 * (it - j * IPT);
-                        const int64_t uu = u + j;
-                        ei = locate(a.ent, e, lv.e0 + lv.ne, uu);
-                        const StackEntry &E = a.ent[ei];
-                        const int s = (int)((uu - E.unit_base) % E.S);
-                        const int k = s * STAGEK + kk;
-                        float v[8];
-                        if (k < E.K) {
-                            load_x8<XBF16, true>(E.x, k, v);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) v[q] = 0.f;
-                        }
-                        float z[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) z[q] = 0.f;
-                        uint2 *st = reinterpret_cast<uint2 *>(bbuf + (size_t)j * FSLOT);
-                        frag_unit<BITS, L>(st, kk, 0, v, a.P, 4, 1, 16, true);
-                        for (int vm = 1; vm * a.P < 4; ++vm) frag_unit<BITS, L>(st, kk, vm, z, a.P, 4, 1, 16, true);
+            // B fragments of tiles [i0, i1) of this level (i relative to u0), one tile per warp
+            // at a time: exact integer digits or bf16 pieces, decided per tile
+            auto build = [&](int i0, int i1) {
+                for (int i = i0 + warp; i < i1; i += kConsumers) {
+                    const Cursor bc = cursor_at(a.ent, lv, u0 + i);
+                    const StackEntry *BE = a.ent + bc.e;
+                    build_slot1<BITS, L, XBF16, true>(bbuf + (size_t)(i - i0) * FSLOT, BE->x, bc.s * STAGEK, BE->K,
+                                                     a.P, lane);
+                }
+            };
+            int chunk_lo = 0, chunk_hi = min(n, a.ucap);
+            build(0, chunk_hi);
+            named_barrier_sync(1, kConsumerThreads);
+
+            Cursor cu = cursor_at(a.ent, lv, u0);
+            const StackEntry *E = a.ent + cu.e;
+            int S = E->S, R = E->R, N = E->N, K = E->K, task_base = E->task_base, spr = E->spr, group = E->group;
+            float *y = E->y;
+            const float *scales = E->scales;
+            int64_t unit_base = E->unit_base;
+            int seg_s0 = cu.s;  // first stage of the current row block in this CTA
+            for (int i = 0; i < n; ++i) {
+                if (i > 0) {
+                    if (cursor_next(cu, S, R)) {
+                        E = a.ent + cu.e;
+                        S = E->S; R = E->R; N = E->N; K = E->K; task_base = E->task_base;
+                        spr = E->spr; group = E->group;
+                        y = E->y;
+                        scales = E->scales;
+                        unit_base = E->unit_base;
                     }
+                    if (cu.s == 0) seg_s0 = 0;
+                }
+                if (i == chunk_hi) {
+                    named_barrier_sync(1, kConsumerThreads);  // every warp is done with the last chunk
+                    chunk_lo = i;
+                    chunk_hi = min(n, i + a.ucap);
+                    build(chunk_lo, chunk_hi);
                     named_barrier_sync(1, kConsumerThreads);
                 }
-                e = locate(a.ent, e, lv.e0 + lv.ne, u);
-                const StackEntry &E = a.ent[e];
-                const int64_t ul = u - E.unit_base;
-                const int rb = (int)(ul / E.S), s = (int)(ul - (int64_t)rb * E.S);
-                const int seg_hi = (E.K * BITS / 8) / (4 * L);  // segments per row
-                const int nsl = min(SPS, seg_hi - s * SPS);
+                const int seg_hi = (K * BITS / 8) / (4 * L);  // segments per row
+                const int nsl = min(SPS, seg_hi - cu.s * SPS);
+                // this lane's scales of the tile (rows pr and pr + 8, the groups of the stage),
+                // read through L1 (a 128-byte line of a row serves many consecutive stages);
+                // their latency overlaps the wait for the tile
+                float s0r[GS], s1r[GS];
+                {
+                    const int gbase = GPS > 0 ? cu.s * GPS : (cu.s * STAGEK) / group;
+                    const int ng = min(GS, spr - gbase);
+                    const float *sp0 = scales + (size_t)min(cu.rb * kSRows + pr, N - 1) * spr + gbase;
+                    const float *sp1 = scales + (size_t)min(cu.rb * kSRows + pr + 8, N - 1) * spr + gbase;
+#pragma unroll
+                    for (int q = 0; q < GS; ++q) {
+                        s0r[q] = q < ng ? __ldg(sp0 + q) : 0.f;
+                        s1r[q] = q < ng ? __ldg(sp1 + q) : 0.f;
+                    }
+                }
                 if (!timed_out) timed_out = !mbar_wait(full + slot, (uint32_t)(round & 1), a.wait_ns);
-                const uint8_t *stg = ring + slot * kTileWords;
+                const uint8_t *stg = ring + slot * kSTile;
                 uint32_t A0[SPS][WPT], A1[SPS][WPT];
 #pragma unroll
                 for (int sl = 0; sl < SPS; ++sl) {
                     lds_words<L>(A0[sl], stg + aoff[sl]);
                     lds_words<L>(A1[sl], stg + aoff[sl] + 8 * kTileBytes);
                 }
-                float s0r[GS], s1r[GS];
-                const float *sc = scl + slot * kTileRows * GS;
-#pragma unroll
-                for (int q = 0; q < GS; ++q) {
-                    s0r[q] = sc[pr * GS + q];
-                    s1r[q] = sc[(pr + 8) * GS + q];
-                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty + slot);  // codes and scales are in registers
+                if (lane == 0) mbar_arrive(empty + slot);  // the codes are in registers
                 if (++slot == kRing) { slot = 0; ++round; }
-                const int64_t cstart = u0 + ((u - u0) / a.ucap) * a.ucap;
-                const uint8_t *fr = bbuf + (size_t)(u - cstart) * FSLOT + fl * 16;
-                if (nsl == SPS)
-                    stage_fixed<BITS, L, 1, 16, GPS, true>(A0, A1, fr, s0r, s1r, nsl, acc);
-                else
-                    stage_fixed<BITS, L, 1, 16, GPS, false>(A0, A1, fr, s0r, s1r, nsl, acc);
+                const uint8_t *slt = bbuf + (size_t)(i - chunk_lo) * FSLOT;
+                const int *hdr = reinterpret_cast<const int *>(slt + slot1_data<BITS>());
+                if (hdr[0]) {
+                    const float fl = digit_lane_factor<BITS>(hdr[1], t);
+                    if (nsl == SPS)
+                        stage1_digits<BITS, L, GPS, true>(A0, A1, slt, lane, s0r, s1r, nsl, fl, ys0, ys1);
+                    else
+                        stage1_digits<BITS, L, GPS, false>(A0, A1, slt, lane, s0r, s1r, nsl, fl, ys0, ys1);
+                } else {
+                    if (nsl == SPS)
+                        stage1_pieces<BITS, L, GPS, true>(A0, A1, slt, lane, s0r, s1r, nsl, ys0, ys1);
+                    else
+                        stage1_pieces<BITS, L, GPS, false>(A0, A1, slt, lane, s0r, s1r, nsl, ys0, ys1);
+                }
 
-                // ---- end of this CTA's share of row block rb ----
-                if (s == E.S - 1 || u == u1 - 1) {
-                    const int T = E.task_base + rb;
-                    const bool whole = (s == E.S - 1) && (u - s >= u0);  // every stage of the row block was here
-                    __syncwarp();
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        redc[pr * 8 + 2 * t + q] = acc[0][q];
-                        redc[(pr + 8) * 8 + 2 * t + q] = acc[0][2 + q];
-                    }
-                    __syncwarp();
-                    if (lane < 16) {
-                        const int r = 16 * warp + lane;
-                        const float *src = redc + r * 8;
-                        float v = src[0];
-                        for (int p = 1; p < a.P; ++p) v += src[p];
-                        if (whole) {
-                            const int n = rb * kTileRows + r;
-                            if (n < E.N) E.y[n] = v;
-                        } else {
-                            // which of this CTA's two partial slots: its first row block, or another
-                            int ef = locate(a.ent, lv.e0, lv.e0 + lv.ne, u0);
-                            const int Tf = a.ent[ef].task_base + (int)((u0 - a.ent[ef].unit_base) / a.ent[ef].S);
-                            a.partial[((size_t)c * 2 + (T == Tf ? 0 : 1)) * kTileRows + r] = v;
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[0][q] = 0.f;
-                    named_barrier_sync(1, kConsumerThreads);
-                    const int64_t tf = E.unit_base + (int64_t)rb * E.S, tl = tf + E.S - 1;
-                    const int cf = cta_of(tf, lv.U, G), clast = cta_of(tl, lv.U, G);
-                    if (ct == 0) {
-                        __threadfence();
-                        if (whole) {
-                            atomicAdd(a.level_done + l, 1);
-                        } else {
-                            int arrivals = 0;
-                            for (int cc = cf; cc <= clast; ++cc) {
-                                int64_t a0, a1;
-                                cta_range(lv.U, cc, G, a0, a1);
-                                arrivals += a0 < a1;
-                            }
-                            const int old = atomicAdd(a.task_cnt + T, 1);
-                            flag[0] = old == arrivals - 1;
-                        }
-                    }
-                    if (!whole) {
-                        named_barrier_sync(1, kConsumerThreads);
-                        if (flag[0]) {
-                            // the last CTA of the row block adds the partial sums in CTA order
+                // ---- end of this CTA's share of row block rb: each warp finishes its 16 rows ----
+                if (cu.s == S - 1 || i == n - 1) {
+                    const int T = task_base + cu.rb;
+                    const bool whole = cu.s == S - 1 && seg_s0 == 0;
+                    // rows pr and pr + 8: the four lanes of each row add their shares
+                    float r0 = ys0 + __shfl_xor_sync(0xffffffffu, ys0, 1);
+                    float r1 = ys1 + __shfl_xor_sync(0xffffffffu, ys1, 1);
+                    r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+                    r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+                    ys0 = ys1 = 0.f;
+                    // lane 4g writes row pr (r0), lane 4g + 1 row pr + 8 (r1)
+                    const int r = pr + 8 * (t & 1);
+                    const float v = (t & 1) ? r1 : r0;
+                    const bool writer = t < 2;
+                    const int nrow = cu.rb * kSRows + r;
+                    if (whole) {
+                        if (writer && nrow < N) y[nrow] = v;
+                        __syncwarp();
+                        if (lane == 0) {
                             __threadfence();
-                            if (ct < kTileRows) {
-                                float v = 0.f;
-                                bool first = true;
-                                for (int cc = cf; cc <= clast; ++cc) {
-                                    int64_t a0, a1;
-                                    cta_range(lv.U, cc, G, a0, a1);
-                                    if (a0 >= a1) continue;
-                                    const int ec = locate(a.ent, lv.e0, lv.e0 + lv.ne, a0);
-                                    const int Tc = a.ent[ec].task_base + (int)((a0 - a.ent[ec].unit_base) / a.ent[ec].S);
-                                    const float pv = ld_cg_f32(a.partial + ((size_t)cc * 2 + (T == Tc ? 0 : 1)) * kTileRows + ct);
-                                    v = first ? pv : v + pv;
-                                    first = false;
+                            atomicAdd(a.level_done + l, 1);
+                        }
+                    } else {
+                        // the partial sums of a CTA's rows go to its slot 0 when the row block
+                        // starts inside the CTA's range, else to slot 1 (a range holds parts of
+                        // at most two split row blocks)
+                        const int64_t tf = unit_base + (int64_t)cu.rb * S;
+                        if (writer) a.partial[((size_t)c * 2 + (u0 >= tf ? 0 : 1)) * kSRows + r] = v;
+                        __syncwarp();
+                        // the CTAs holding parts of this row block (lanes take one each), and
+                        // whether this warp is the last of them to arrive for its rows
+                        const int cf = cta_of(tf, lv.U, G), clast = cta_of(tf + S - 1, lv.U, G);
+                        int arrivals = 0;
+                        for (int base = cf; base <= clast; base += 32) {
+                            const int cc = base + lane;
+                            const bool in = cc <= clast && us[cc] < us[cc + 1];
+                            arrivals += __popc(__ballot_sync(0xffffffffu, in));
+                        }
+                        int last = 0;
+                        if (lane == 0) {
+                            __threadfence();
+                            last = atomicAdd(a.task_cnt + (size_t)T * kConsumers + warp, 1) == arrivals - 1;
+                        }
+                        last = __shfl_sync(0xffffffffu, last, 0);
+                        if (last) {
+                            // lane j reads the 16 partial sums of CTA cf + j; the warp adds them
+                            // in a fixed tree order (deterministic), 32 CTAs at a time in order;
+                            // lane rr keeps row 16 * warp + rr
+                            __threadfence();
+                            float mine = 0.f;
+                            for (int base = cf; base <= clast; base += 32) {
+                                const int cc = base + lane;
+                                const bool in = cc <= clast && us[cc] < us[cc + 1];
+                                float pv[16];
+                                if (in) {
+                                    const float4 *src = reinterpret_cast<const float4 *>(
+                                        a.partial + ((size_t)cc * 2 + (us[cc] >= tf ? 0 : 1)) * kSRows + 16 * warp);
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        const float4 f4 = __ldcg(src + q);
+                                        pv[4 * q] = f4.x; pv[4 * q + 1] = f4.y; pv[4 * q + 2] = f4.z; pv[4 * q + 3] = f4.w;
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int q = 0; q < 16; ++q) pv[q] = 0.f;
                                 }
-                                const int n = rb * kTileRows + ct;
-                                if (n < E.N) E.y[n] = v;
+#pragma unroll
+                                for (int rr = 0; rr < 16; ++rr) {
+                                    float t2 = pv[rr];
+#pragma unroll
+                                    for (int m = 16; m >= 1; m >>= 1) t2 += __shfl_xor_sync(0xffffffffu, t2, m);
+                                    if (lane == rr) mine = base == cf ? t2 : mine + t2;
+                                }
                             }
-                            named_barrier_sync(1, kConsumerThreads);
-                            if (ct == 0) {
-                                a.task_cnt[T] = 0;
+                            const int nr = cu.rb * kSRows + 16 * warp + lane;
+                            if (lane < 16 && nr < N) y[nr] = mine;
+                            __syncwarp();
+                            if (lane == 0) {
+                                a.task_cnt[(size_t)T * kConsumers + warp] = 0;
                                 __threadfence();
                                 atomicAdd(a.level_done + l, 1);
                             }
@@ -379,10 +422,10 @@ __global__ void __maxnreg__(96) gemv_stack(const StackArgs a) {
             }
         }
     }
-    if (timed_out) flag[1] = 1;
+    if (timed_out) flag[0] = 1;
     __syncthreads();
     if (threadIdx.x == 0) {
-        if (flag[1]) {
+        if (flag[0]) {
             if (a.status) atomicOr(a.status, Q4_STATUS_TIMEOUT);
             atomicExch(a.tflag, 1);
         }
@@ -393,7 +436,7 @@ __global__ void __maxnreg__(96) gemv_stack(const StackArgs a) {
             __threadfence();
             for (int l = 0; l < a.L; ++l) a.level_done[l] = 0;
             if (atomicAdd(a.tflag, 0)) {
-                for (int i = 0; i < a.n_tasks; ++i) a.task_cnt[i] = 0;
+                for (int i = 0; i < a.n_tasks * kConsumers; ++i) a.task_cnt[i] = 0;
                 *a.tflag = 0;
             }
             *a.finished = 0;
@@ -435,7 +478,7 @@ bool stack_format(int bits, int64_t K, int64_t group, int *L, int *gps) {
 
 struct StackLayout {
     int L, gps, nlev, n_tasks;
-    size_t off_ent, off_lev, off_cnt, off_done, off_misc, off_part, bytes;
+    size_t off_ent, off_lev, off_cnt, off_done, off_misc, off_part, off_us, bytes;
 };
 
 q4_status stack_layout(const q4_stack_gemv *gv, int32_t count, int bits, q4_xdtype xt, StackLayout *lo) {
@@ -456,7 +499,7 @@ q4_status stack_layout(const q4_stack_gemv *gv, int32_t count, int bits, q4_xdty
         } else if (L != lo->L || gps != lo->gps) {
             return Q4_ERR_UNSUPPORTED;  // one kernel variant per stack
         }
-        tasks += (g.N + kTileRows - 1) / kTileRows;
+        tasks += (g.N + kSRows - 1) / kSRows;
     }
     if (tasks > (int64_t)1 << 30) return Q4_ERR_UNSUPPORTED;
     lo->nlev = gv[count - 1].level + 1;
@@ -464,10 +507,11 @@ q4_status stack_layout(const q4_stack_gemv *gv, int32_t count, int bits, q4_xdty
     lo->off_ent = 0;
     lo->off_lev = al256((size_t)count * sizeof(StackEntry));
     lo->off_cnt = lo->off_lev + al256((size_t)lo->nlev * sizeof(StackLevel));
-    lo->off_done = lo->off_cnt + al256((size_t)lo->n_tasks * 4);
+    lo->off_done = lo->off_cnt + al256((size_t)lo->n_tasks * kConsumers * 4);
     lo->off_misc = lo->off_done + al256((size_t)lo->nlev * 4);
     lo->off_part = lo->off_misc + 256;
-    lo->bytes = lo->off_part + al256((size_t)kPlanGrid * 2 * kTileRows * 4);
+    lo->off_us = lo->off_part + al256((size_t)kPlanGrid * 2 * kSRows * 4);
+    lo->bytes = lo->off_us + al256((size_t)lo->nlev * (kPlanGrid + 1) * 4);
     return Q4_OK;
 }
 
@@ -541,7 +585,7 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
             const q4_stack_gemv &g = gemvs[i];
             StackEntry &E = ent[i];
             std::memset(&E, 0, sizeof E);
-            if (!encode_payload_map(&E.tm, g.payload, g.N, g.K, bits)) return Q4_ERR_UNSUPPORTED;
+            if (!encode_payload_map(&E.tm, g.payload, g.N, g.K, bits, kSRows)) return Q4_ERR_UNSUPPORTED;
             E.scales = g.scales;
             E.x = g.x;
             E.y = g.y;
@@ -550,7 +594,7 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
             E.group = (int)g.group;
             E.spr = (int)(g.K / g.group);
             E.S = (int)((g.K * bits / 8 + kTileBytes - 1) / kTileBytes);
-            E.R = (int)((g.N + kTileRows - 1) / kTileRows);
+            E.R = (int)((g.N + kSRows - 1) / kSRows);
             E.task_base = task_base;
             E.level = l;
             E.unit_base = lv.U;
@@ -562,12 +606,9 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     }
 
     // shared memory and grid
-    const int stagek = kTileBytes * 8 / bits;
-    const int kts = stagek / 16;
-    const size_t fslot = (size_t)kts * 16 * 8;
+    const size_t fslot = bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>();  // B fragments + header of a tile
     const int gsl = lo.gps > 0 ? lo.gps : 1;
-    const size_t fixed = 1024 + (size_t)kRing * kTileWords + (size_t)kRing * kTileRows * gsl * 4 +
-                         (size_t)kTileRows * 8 * 4 + 2 * kRing * 8 + 16;
+    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16;
     if (fixed + fslot > (size_t)kSmemBudget) return Q4_ERR_UNSUPPORTED;
     int ucap = (int)((kSmemBudget - fixed) / fslot);
     if (ucap > 64) ucap = 64;
@@ -584,12 +625,20 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     int grid = sms * (per_sm < kCtasPerSm ? per_sm : kCtasPerSm);
     if (grid > kPlanGrid) grid = kPlanGrid;
 
+    // each CTA's first tile in each level: an even split of the level's tiles
+    std::vector<int> ustart((size_t)lo.nlev * (grid + 1));
+    for (int l = 0; l < lo.nlev; ++l) {
+        if (lev[l].U >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
+        for (int cc = 0; cc <= grid; ++cc) ustart[(size_t)l * (grid + 1) + cc] = (int)(lev[l].U * cc / grid);
+    }
     // copy the tables, zero the counters; the host tables can go once the stream is done
     char *w = static_cast<char *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((e = cudaMemcpyAsync(w + lo.off_ent, ent.data(), ent.size() * sizeof(StackEntry), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(w + lo.off_lev, lev.data(), lev.size() * sizeof(StackLevel), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(w + lo.off_us, ustart.data(), ustart.size() * sizeof(int), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
         (e = cudaMemsetAsync(w + lo.off_cnt, 0, lo.off_part - lo.off_cnt, s)) != cudaSuccess ||
         (e = cudaStreamSynchronize(s)) != cudaSuccess)
@@ -605,6 +654,7 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     p.args.finished = reinterpret_cast<int *>(w + lo.off_misc);
     p.args.tflag = reinterpret_cast<int *>(w + lo.off_misc) + 1;
     p.args.partial = reinterpret_cast<float *>(w + lo.off_part);
+    p.args.ustart = reinterpret_cast<const int *>(w + lo.off_us);
     p.args.status = nullptr;
     p.args.G = grid;
     p.args.L = lo.nlev;

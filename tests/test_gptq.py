@@ -118,6 +118,24 @@ def test_errors(q4):
     assert lib.q4_gptq_quantize(None, 0, 8, None, 4, 8, None, None, 0) == q4.Q4_OK  # N = 0: nothing to do
 
 
+def test_ill_conditioned_U_reports_nonfinite_and_leaves_outputs(q4):
+    # a tiny diagonal with large off-diagonal entries makes the error feedback grow past the
+    # fp32 range: the call reports it and writes neither payload nor scales
+    import ctypes
+
+    K, N = 64, 4
+    U = np.triu(np.full((K, K), 1e30))
+    np.fill_diagonal(U, 1e-30)
+    w = np.random.default_rng(0).normal(0, 1, (N, K)).astype(np.float32)
+    payload = np.full(N * K // 2, 0xAB, np.uint8)
+    scales = np.full(N * K // 32, -7.0, np.float32)
+    vp = ctypes.c_void_p
+    st = q4.lib().q4_gptq_quantize(w.ctypes.data_as(vp), N, K, U.ctypes.data_as(vp), 4, 32,
+                                   payload.ctypes.data_as(vp), scales.ctypes.data_as(vp), 2)
+    assert st == q4.Q4_ERR_NONFINITE
+    assert np.all(payload == 0xAB) and np.all(scales == -7.0)
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("bits,group", [(4, 128), (8, 512)])
 def test_gptq_payload_runs_through_qgemm(q4, bits, group):

@@ -167,7 +167,8 @@ def test_bf16_activations(q4, M):
 
 
 def test_activation_range_extremes(q4):
-    # tiny, huge and mixed-magnitude activations: the exact fp16 split rescales by 2^-e
+    # tiny, huge and mixed-magnitude activations: each activation is split exactly into
+    # three bf16 pieces, so every product keeps its own exponent
     rng = np.random.default_rng(5)
     w = rng.normal(0, 0.02, (64, 512)).astype(np.float32)
     for scale in (1e-30, 1e-8, 1e-3, 1e4, 1e30):

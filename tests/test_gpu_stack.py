@@ -224,3 +224,43 @@ def test_llama7b_stack_sampled(q4):
         y = g.y.cpu().numpy()[rows].astype(np.float64).reshape(1, -1)
         err = np.abs(y - yref)
         assert np.all(err <= RTOL * bound + ATOL), f"GEMV {idx}: worst ratio {(err / (RTOL * bound + ATOL)).max():.3g}"
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_stages_of_every_activation_range(q4, bits):
+    # per 128-byte stage the kernel takes exact integer digits when the stage's activations
+    # span at most 2^21, else exact bf16 pieces: stages of ordinary, zero, tiny, huge and
+    # adversarial activations (one 1e7 on a column of zero codes) side by side, in a
+    # two-level stack whose second level reads the first one's output
+    import torch
+
+    rng = np.random.default_rng(11 + bits)
+    stagek = 256 if bits == 4 else 128
+    K, N = 12 * stagek, 640
+    x = rng.normal(0, 1, K).astype(np.float32)
+    st = lambda i: slice(i * stagek, (i + 1) * stagek)
+    x[st(1)] = 0.0                                      # all zero
+    x[st(2)] *= np.float32(1e-30)                        # tiny
+    x[st(3)] *= np.float32(1e30)                         # huge
+    x[st(4)][::3] *= np.float32(2.0 ** -20)               # range just inside 2^21
+    x[st(5)][::3] *= np.float32(2.0 ** -23)               # range just outside
+    zero_col = 6 * stagek + 17
+    x[zero_col] = 1e7                                   # huge activation on a zero-code column
+    x[st(7)][::5] = 0.0                                  # exact zeros among normal values
+    x[st(8)] = x[st(8)].astype(np.float32) * np.float32(3e-20)
+    w = rng.normal(0, 1 / np.sqrt(K), (N, K)).astype(np.float32)
+    w[:, zero_col] = 0.0
+    w2 = rng.normal(0, 1 / np.sqrt(N), (N, N)).astype(np.float32)
+    p, s, _ = oracle.pack(w, bits, 128)
+    p2, s2, _ = oracle.pack(w2, bits, 128)
+    xd = torch.from_numpy(x).cuda()
+    y1 = torch.empty(N, device="cuda")
+    y2 = torch.empty(N, device="cuda")
+    gemvs = [q4.StackGemv(torch.from_numpy(p).cuda(), torch.from_numpy(s).cuda(), xd, y1, N, K, 128, 0),
+             q4.StackGemv(torch.from_numpy(p2).cuda(), torch.from_numpy(s2).cuda(), y1, y2, N, N, 128, 1)]
+    stack = q4.DecodeStack(gemvs, bits)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stack.run(status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check_all(gemvs, [("w", 0, N, K, 128, p, s), ("w2", 0, N, N, 128, p2, s2)], bits, f"ranges int{bits}")
