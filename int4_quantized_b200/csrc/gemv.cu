@@ -116,11 +116,19 @@ Q4_DEVINL int stored_cols(int NB, int lw) { return (lw == 16 ? 4 : 8) * NB; }
 
 // One CTA per (k-block eb, 16-row chunk mc of x): the pieces of the block in MMA order
 // (several rows of x), zero columns for rows past M.
-template <int BITS, int L, bool XBF16>
+template <int BITS, int L, bool XBF16, bool HYB>
 __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
     grid_dep_launch();
     grid_dep_wait();  // x may be the output of the kernel before this one
     constexpr int STAGEK = kTileBytes * 8 / BITS;
+    if constexpr (HYB) {
+        // one row of x: each warp builds whole stage slots of the k-block (digits or pieces)
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int s0 = blockIdx.x * a.ebs, s1 = min(s0 + a.ebs, a.stages_total);
+        for (int s = s0 + warp; s < s1; s += 8)
+            build_slot1<BITS, L, XBF16, false>(a.frag + (size_t)s * a.fslot_bytes, a.x, s * STAGEK, a.K, a.P, lane);
+        return;
+    }
     const int eb = blockIdx.x, mc = blockIdx.y;
     const int mcnt = min(16, a.M - mc * 16);
     const int ncols = stored_cols(a.NB, a.lw);
@@ -149,7 +157,7 @@ __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
 // otherwise the pieces come from gemv_prep through a second ring. GPS: groups per stage
 // when they divide it, 0 when the stage lies inside one group, -1 for any other group
 // size (tracked segment by segment at run time).
-template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16>
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB>
 __global__ void __launch_bounds__(kThreads) __maxnreg__(NB >= 3 ? 160 : 96)
 gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     constexpr int SPS = kTileBytes / (4 * L);          // segments per stage
@@ -160,6 +168,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     constexpr bool PAIRED = NB <= 2;
     constexpr int LW = INK ? 16 : 32;  // piece lanes stored per (MMA, n8 block), workspace: a.lw
     static_assert(!INK || NB == 1, "on-chip pieces cover one row of x");
+    static_assert(!HYB || (NB == 1 && GPS >= 0), "one row of x, regular groups");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int nring = a.nst_ring;
@@ -313,7 +322,14 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         // x may be the output of the kernel before this one, and y may still be read by it
         // (a no-op unless this grid was launched as a dependent)
         grid_dep_wait();
-        if constexpr (INK) {
+        if constexpr (INK && HYB) {
+            // the B fragments of this CTA's stages (digits or pieces, per stage), one stage
+            // per warp, built while the first payload tiles are in flight
+            for (int ls = warp; ls < nst; ls += kConsumers)
+                build_slot1<BITS, L, XBF16, false>(fslots + (size_t)ls * a.fslot_bytes, a.x, (st_lo + ls) * STAGEK,
+                                                  a.K, a.P, lane);
+            named_barrier_sync(1, kConsumerThreads);
+        } else if constexpr (INK) {
             // pieces of this CTA's K range of the single activation row, built while the
             // first payload tiles are in flight; column 3 (and the 16 lanes above, which
             // repeat these) is zero
@@ -347,6 +363,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
         }
         const int lwr = INK ? LW : a.lw;
         const int fl = lane & (lwr - 1);  // lanes past the stored width repeat lanes (their columns are unused)
+        float ys0 = 0.f, ys1 = 0.f;  // one row of x: this lane's share of rows pr and pr + 8
         float cacc[NB][4], acc[NB][4];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -403,7 +420,23 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                 if (!timed_out) timed_out = !mbar_wait(ffull + slot, (uint32_t)(round & 1));
                 fr = fslots + slot * a.fslot_bytes;
             }
-            if constexpr (GPS >= 0) {
+            if constexpr (HYB) {
+                const int qb = (GPS > 0 ? s * GPS : (s * SPS) / a.spg) - gA;  // first group, in the k-block
+                const float *s0p = sb + pr * kSG + qb, *s1p = s0p + 8 * kSG;
+                const int *hdr = reinterpret_cast<const int *>(fr + slot1_data<BITS>());
+                if (hdr[0]) {
+                    const float fl8 = digit_lane_factor<BITS>(hdr[1], t);
+                    if (nsl == SPS)
+                        stage1_digits<BITS, L, GPS, true>(A0, A1, fr, lane, s0p, s1p, nsl, fl8, ys0, ys1);
+                    else
+                        stage1_digits<BITS, L, GPS, false>(A0, A1, fr, lane, s0p, s1p, nsl, fl8, ys0, ys1);
+                } else {
+                    if (nsl == SPS)
+                        stage1_pieces<BITS, L, GPS, true>(A0, A1, fr, lane, s0p, s1p, nsl, ys0, ys1);
+                    else
+                        stage1_pieces<BITS, L, GPS, false>(A0, A1, fr, lane, s0p, s1p, nsl, ys0, ys1);
+                }
+            } else if constexpr (GPS >= 0) {
                 const int qb = (GPS > 0 ? s * GPS : (s * SPS) / a.spg) - gA;  // first group, in the k-block
                 const float *s0p = sb + pr * kSG + qb, *s1p = s0p + 8 * kSG;
                 const uint8_t *frl = fr + fl * (PAIRED ? 16 : 8);
@@ -455,6 +488,24 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             }
             if (++slot == nring) { slot = 0; ++round; }
         }
+        if constexpr (HYB) {
+            // one row of x: the four lanes of each row add their shares; lane 4g writes row
+            // pr, lane 4g + 1 row pr + 8 (the partial sums of a K split go to the ring,
+            // which every warp must be done with first)
+            float r0 = ys0 + __shfl_xor_sync(0xffffffffu, ys0, 1);
+            float r1 = ys1 + __shfl_xor_sync(0xffffffffu, ys1, 1);
+            r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+            r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+            const int r = pr + 8 * (t & 1);
+            const float v = (t & 1) ? r1 : r0;
+            if (a.CS == 1) {
+                const int n = cl * kRowsPerCta + r;
+                if (t < 2 && n < a.N) a.y[n] = v;
+            } else {
+                named_barrier_sync(1, kConsumerThreads);
+                if (t < 2) red[r * 16] = v;
+            }
+        } else {
         // add the pieces of each activation row: every warp writes its rows' piece columns
         // (column P * m + p) and sums its own rows; the ring is reused, so every warp must
         // be done with it first
@@ -479,6 +530,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             } else {
                 red[r * 16 + m] = v;
             }
+        }
         }
     }
     if (timed_out && a.status) atomicOr(a.status, Q4_STATUS_TIMEOUT);
@@ -508,7 +560,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
 // early: the weights are static, so the call's first grid may start (and the stream
 // kernel read payload and scales) while the previous kernel on the stream still runs.
 // Every read of x, and every write, still waits for that kernel to finish.
-template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16>
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB = false>
 cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
                          bool early, cudaStream_t st) {
     cudaError_t err;
@@ -525,11 +577,11 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
         pc.stream = st;
         pc.attrs = &pdl;
         pc.numAttrs = early ? 1 : 0;
-        err = x_bf16 ? cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, true>, a)
-                     : cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, false>, a);
+        err = x_bf16 ? cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, true, HYB>, a)
+                     : cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, false, HYB>, a);
         if (err != cudaSuccess) return err;
     }
-    auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16>;
+    auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16, HYB>;
     const size_t smem = pl.smem_bytes;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
@@ -558,10 +610,17 @@ cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorM
                           bool early, cudaStream_t st) {
 #define Q4_INK(B, LL, G)                                                                         \
     if (pl.bits == B && pl.L == LL && pl.gps == G)                                               \
-        return x_bf16 ? launch_typed<B, LL, 1, G, true, true>(pl, a, tm, true, early, st)        \
-                      : launch_typed<B, LL, 1, G, true, false>(pl, a, tm, false, early, st);
+        return x_bf16 ? launch_typed<B, LL, 1, G, true, true, (G >= 0)>(pl, a, tm, true, early, st) \
+                      : launch_typed<B, LL, 1, G, true, false, (G >= 0)>(pl, a, tm, false, early, st);
 #define Q4_STAGED(B, LL, G)                                                                      \
     if (pl.bits == B && pl.L == LL && pl.gps == G) {                                             \
+        if (pl.hyb) {                                                                            \
+            if constexpr (G >= 0)                                                                \
+                return x_bf16 ? launch_typed<B, LL, 1, (G >= 0 ? G : 0), false, true, true>(      \
+                                    pl, a, tm, true, early, st)                                  \
+                              : launch_typed<B, LL, 1, (G >= 0 ? G : 0), false, false, true>(     \
+                                    pl, a, tm, false, early, st);                                \
+        }                                                                                        \
         switch (pl.NB) {                                                                         \
             case 1: return launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, early, st); \
             case 2: return launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, early, st); \
@@ -663,10 +722,12 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, bool x_
     p.CS = cs < 1 ? 1 : (int)cs;
     p.stages_per_cta = (p.stages_total + p.CS - 1) / p.CS;
     const int kts = bits == 4 ? 16 : 8;  // MMAs per stage
-    // one row of x: 16 piece lanes, built on chip when the CTA's K range fits
+    // one row of x: 16 piece lanes, built on chip when the CTA's K range fits; with
+    // regular groups each stage's slot holds digits or pieces plus a header
     p.ink = M == 1 && (int64_t)p.stages_per_cta * stagek <= kInkMaxK;
     if (p.ink) p.lw = 16;
-    p.fslot_bytes = kts * p.NB * p.lw * 8;
+    p.hyb = M == 1 && p.gps >= 0;
+    p.fslot_bytes = p.hyb ? (bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>()) : kts * p.NB * p.lw * 8;
     const size_t fixed = 1024 + 2 * (size_t)kRowsPerCta * kSG * 4 + (4 * kMaxStages + 4) * 8;
     int nr;
     if (p.ink) {

@@ -41,6 +41,7 @@ struct GemvPlan {
     int nst_ring;       // ring depth
     int fslot_bytes;    // piece bytes of one stage
     int ink;            // one row of x: pieces built in shared memory, no workspace
+    int hyb;            // one row of x, regular groups: per stage, exact digits or pieces
     int nmc;            // 16-row chunks of x = ceil(M / 16)
     size_t smem_bytes;  // dynamic shared memory per CTA
     size_t off_frag, bytes;  // workspace layout and size (0 when ink)

@@ -100,10 +100,16 @@ Q4_DEVINL int ld_acquire(const int *p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-Q4_DEVINL float ld_cg_f32(const float *p) {
-    float v;
-    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
-    return v;
+// Counter updates that publish (release) everything this warp wrote before them (the
+// __syncwarp() before each call orders the other lanes' writes first); the acquire-release
+// form also makes every write published before the value it reads visible to the warp.
+Q4_DEVINL void red_release_add(int *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+Q4_DEVINL int atom_acq_rel_add(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 Q4_DEVINL void tmap_acquire(const CUtensorMap *tm) {
     asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(tm) : "memory");
@@ -245,10 +251,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             if (l > 0) {
                 // the activations of this level are complete once every warp of every row
                 // block of the previous level has published its rows
-                if (ct == 0 && !timed_out) {
+                if (ct == 0 && !timed_out)
                     timed_out = !wait_counter(a.level_done + (l - 1), kConsumers * a.lev[l - 1].T, a.wait_ns);
-                    __threadfence();
-                }
                 named_barrier_sync(1, kConsumerThreads);
             }
             // B fragments of tiles [i0, i1) of this level (i relative to u0), one tile per warp
@@ -352,10 +356,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                     if (whole) {
                         if (writer && nrow < N) y[nrow] = v;
                         __syncwarp();
-                        if (lane == 0) {
-                            __threadfence();
-                            atomicAdd(a.level_done + l, 1);
-                        }
+                        if (lane == 0) red_release_add(a.level_done + l, 1);
                     } else {
                         // the partial sums of a CTA's rows go to its slot 0 when the row block
                         // starts inside the CTA's range, else to slot 1 (a range holds parts of
@@ -373,16 +374,14 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                             arrivals += __popc(__ballot_sync(0xffffffffu, in));
                         }
                         int last = 0;
-                        if (lane == 0) {
-                            __threadfence();
-                            last = atomicAdd(a.task_cnt + (size_t)T * kConsumers + warp, 1) == arrivals - 1;
-                        }
+                        if (lane == 0)
+                            last = atom_acq_rel_add(a.task_cnt + (size_t)T * kConsumers + warp, 1) == arrivals - 1;
                         last = __shfl_sync(0xffffffffu, last, 0);
                         if (last) {
                             // lane j reads the 16 partial sums of CTA cf + j; the warp adds them
                             // in a fixed tree order (deterministic), 32 CTAs at a time in order;
                             // lane rr keeps row 16 * warp + rr
-                            __threadfence();
+                            __syncwarp();
                             float mine = 0.f;
                             for (int base = cf; base <= clast; base += 32) {
                                 const int cc = base + lane;
@@ -413,8 +412,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                             __syncwarp();
                             if (lane == 0) {
                                 a.task_cnt[(size_t)T * kConsumers + warp] = 0;
-                                __threadfence();
-                                atomicAdd(a.level_done + l, 1);
+                                red_release_add(a.level_done + l, 1);
                             }
                         }
                     }
