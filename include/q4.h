@@ -118,15 +118,14 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
                    int bits, int64_t group, float *w_out, void *stream);
 
 /*
- * Workspace bytes that qgemm needs for this problem: with two or more rows of
- * x, the activations converted once into fixed-point digits in tensor-core
- * fragment order (4 bytes per element of x, rows padded to pairs and 16-row
- * chunks) plus one exponent per row of x and block of up to 1024 k. One row
- * of x needs none (0) when each CTA's share of K fits on chip, which holds up
- * to K = 8192 per CTA. Groups of whole rows (group a multiple of K) add N
- * floats, rounded up to 256 bytes, at the start: their scales spread to one
- * per row. Same arguments as qgemm. Returns 0 for arguments qgemm rejects.
- * Depends only on the arguments, not on the device.
+ * Workspace bytes that qgemm needs for this problem: the activations converted once
+ * into tensor-core fragments (exact bf16 pieces, 3 per fp32 activation, in MMA order;
+ * for one row of x, per 128-byte stage either those pieces or exact 40-bit fixed-point
+ * digits, 2064 bytes per int4 stage and 1040 per int8 stage). One row of x needs none (0)
+ * when each CTA's share of K, at most 4096, is built on chip. Groups of whole rows
+ * (group a multiple of K) add N floats, rounded up to 256 bytes, at the start: their
+ * scales spread to one per row. Same arguments as qgemm. Returns 0 for arguments qgemm
+ * rejects. Depends only on the arguments, not on the device.
  */
 Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt);
@@ -151,8 +150,12 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  *            caller zeroes it and reads it after synchronizing the stream.
  * Paths: M <= 63, or fp32 x at any M: the fused unpack->dequant->GEMV kernel
  * (rows of x in chunks of 16). bf16 x with M >= 64: the tensor-core GEMM.
- * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for
- * finite inputs (y_exact = the fp64 sum).
+ * Accuracy: |y - y_exact| <= 1e-5 * sum_k |w'[n][k] x[m][k]| + 1e-6 for every
+ * finite x (y_exact = the fp64 sum), however widely the magnitudes of x spread: the
+ * codes enter the tensor cores exactly; the activations enter as three exact bf16
+ * pieces, or (one row of x, a 128-byte stage whose activations span at most 2^21)
+ * as fixed-point digits within 2^-18 of each activation's own magnitude; the sums
+ * are fp32. Activations below 2^-110 in magnitude may lose bits below 2^-133.
  * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0; group divides K with
  * group % 32 == 0 (per-channel scales are group = K), or group is a multiple
  * of K (groups of whole rows, down to one scale for the whole matrix, the
