@@ -520,21 +520,14 @@ Q4_DEVINL void stage1_digits(const uint32_t (&A0)[kTileBytes / (4 * L)][L / 4],
     }
 }
 
-// Builds the slot of one stage from its activations x[k0, k0 + STAGEK) (zeros past K): the
-// calling warp's lanes take 8 k each (all 32 for int4, 16 for int8), decide the format
-// together and write every byte of the slot (header by lane 0).
-template <int BITS, int L, bool XBF16, bool CG>
-Q4_DEVINL void build_slot1(uint8_t *slot, const void *x, int k0, int K, int P, int lane) {
+// Builds the slot of one stage from the calling lane's 8 activations v (k = 8 * lane + q
+// of the stage; zeros past K and in lanes past the stage): the warp decides the format
+// together and writes every byte of the slot (header by lane 0).
+template <int BITS, int L>
+Q4_DEVINL void build_slot1_v(uint8_t *slot, const float (&v)[8], int P, int lane) {
     constexpr int STAGEK = kTileBytes * 8 / BITS;
     constexpr int LANES = STAGEK / 8;
     const int kk = 8 * lane;
-    float v[8];
-    if (lane < LANES && k0 + kk < K) {
-        load_x8<XBF16, CG>(x, k0 + kk, v);
-    } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = 0.f;
-    }
     uint32_t mx = 0, mn = 0x7f800000u;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -558,6 +551,23 @@ Q4_DEVINL void build_slot1(uint8_t *slot, const void *x, int k0, int K, int P, i
         h[0] = dig ? 1 : 0;
         h[1] = E;
     }
+}
+
+// The same from x[k0, k0 + STAGEK) in global memory (zeros past K): the calling warp's
+// lanes load 8 k each (all 32 for int4, 16 for int8).
+template <int BITS, int L, bool XBF16, bool CG>
+Q4_DEVINL void build_slot1(uint8_t *slot, const void *x, int k0, int K, int P, int lane) {
+    constexpr int STAGEK = kTileBytes * 8 / BITS;
+    constexpr int LANES = STAGEK / 8;
+    const int kk = 8 * lane;
+    float v[8];
+    if (lane < LANES && k0 + kk < K) {
+        load_x8<XBF16, CG>(x, k0 + kk, v);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = 0.f;
+    }
+    build_slot1_v<BITS, L>(slot, v, P, lane);
 }
 
 // The lane's multiplier of the digits format: 2^(E - 38) times its column pair's weight

@@ -10,18 +10,27 @@
 //     when the level starts (the outputs of earlier levels, or inputs given by the
 //     caller); level l + 1 may read what level l writes (q/k/v, then o, then gate/up,
 //     then down, in a transformer layer).
-//   * The weight tiles (128 rows x 128 bytes) of a level are numbered GEMV by GEMV, row
+//   * The weight tiles (240 rows x 128 bytes) of a level are numbered GEMV by GEMV, row
 //     block by row block, k-stage by k-stage, and each of the G resident CTAs takes one
 //     contiguous G-th of them (an even split of the level's bytes, whatever its shapes).
 //   * A producer warp per CTA streams the CTA's tiles of every level, in order, through
-//     one TMA ring, with the scales of each tile beside it. It never waits for a level:
-//     the weights are static, so the next level's tiles arrive while the current level
-//     ends and its activations are published.
-//   * Eight consumer warps wait (bounded, on a device counter) until the previous level
-//     is complete, build the bf16 pieces of x for their tiles, and multiply. A row block
-//     whose k-stages were split over several CTAs is added up by whichever CTA finishes
-//     its share last, from the partial sums in fixed CTA order (deterministic results).
-//     A completed row block increments the level's counter.
+//     one TMA ring, and asks L2 for the scales each stretch of tiles will need. It never
+//     waits for a level: the weights are static, so the next level's tiles arrive while
+//     the current level ends.
+//   * Fifteen consumer warps (16 rows of each tile apiece) wait (bounded, on a device
+//     counter) until every part of the previous level is published, build the exact
+//     digits or bf16 pieces of x for their tiles, and multiply.
+//   * A row block whose k-stages fall to several CTAs ends as several parts, one per
+//     CTA, kept in a [parts][rows] matrix per GEMV; a part is published with one release
+//     increment of the level's counter, without waiting for the other parts. Nobody
+//     adds the parts up on the way to the next level: where a GEMV's x is a slice of a
+//     previous-level GEMV's y, the next level reads x as the sum of that slice's parts
+//     (in part order; absent parts are zeros). The y of a split row block is written by
+//     the CTA holding its last part, as the same sum, so y and what the next level read
+//     are the same numbers; it does so at the start of the level after next, while it
+//     waits for the level before to end (at the next start if the next level reads that
+//     y directly). A level waits for the sums of three levels back (the parts buffers
+//     rotate over three levels) and of every earlier level whose y it reads directly.
 //   * Counters return to zero at the end of every launch (the last CTA to finish resets
 //     them), so the workspace can be replayed, e.g. from a CUDA graph.
 //
@@ -30,6 +39,7 @@
 // producer waits (bounded) for every copy it issued into the CTA's shared memory.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstring>
 #include <vector>
 
@@ -57,41 +67,47 @@ constexpr int kSmemBudget = 163840;
 constexpr int kCtasPerSm = 1;
 
 struct alignas(64) StackEntry {
-    CUtensorMap tm;        // 2D map of the payload: {row bytes, N}, box 128 x 128, 128B swizzle
+    CUtensorMap tm;        // 2D map of the payload: {row bytes, N}, box 128 x 240, 128B swizzle
+    // consumer fields (one 128-byte line)
     const float *scales;
     const void *x;
     float *y;
+    float *parts;          // [pmax][npad] the parts of this GEMV's row blocks
+    const float *xparts;   // non-null: x is the sum over xpmax parts of these rows (stride xstride)
     int64_t unit_base;     // first tile of this GEMV in its level's numbering
     int N, K;
     int group;             // scale group (divides K)
     int spr;               // scales per row = K / group
     int S;                 // k-stages per row (128 bytes of payload each)
-    int R;                 // row blocks of 128
-    int task_base;         // global index of row block 0
+    int R;                 // row blocks of 240
+    int pmax, npad;        // parts per row block at most; row stride of parts
+    int xpmax, xstride;
+    int is_src;            // the next level reads x from this GEMV's parts
     int level;
 };
 
 struct StackLevel {
     int64_t U;             // tiles in the level
     int e0, ne;            // its GEMVs
-    int T;                 // row blocks in the level
-    int pad;
+    int parts_target;      // arrivals that complete the level: 15 per (row block, part)
+    int fin_target;        // arrivals that complete its sums of split row blocks: one per block
+    int fin_lo, fin_hi;    // levels whose sums must be in y before this level starts (none: lo > hi)
+    int needs_final;       // it reads a y of the previous level other than as a slice of parts
+    int fin_early;         // the next level reads its y other than as parts: sums at the next start
 };
 
 struct StackArgs {
     const StackEntry *ent;
     const StackLevel *lev;
-    int *task_cnt;         // [n_tasks][15] arrivals of the CTAs sharing a row block, per warp
-    int *level_done;       // [L] completed (row block, warp) pairs per level
+    int *parts_done;       // [L] published (row block, part, warp) triples per level
+    int *fin_done;         // [L] finished (split row block, warp) sums per level
     int *finished;         // CTAs done with the launch
-    int *tflag;            // set when a wait gave up: the last CTA also resets task_cnt
-    float *partial;        // [G][2][240] partial sums
     const int *ustart;     // [L][G + 1] first tile of each CTA's range in each level
+    const int *pfirst;     // [L][G] part index of the row block each CTA's range starts in
     uint32_t *status;
-    int G, L, n_tasks;
+    int G, L;
     int P;                 // pieces per activation: 3 (fp32 x) or 1 (bf16 x)
     int ucap;              // tiles whose activation pieces fit in shared memory at once
-    int gs;                // scale slots per row per tile (max(1, groups per tile))
     uint64_t wait_ns;      // bound of every wait
 };
 
@@ -100,16 +116,10 @@ Q4_DEVINL int ld_acquire(const int *p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Counter updates that publish (release) everything this warp wrote before them (the
-// __syncwarp() before each call orders the other lanes' writes first); the acquire-release
-// form also makes every write published before the value it reads visible to the warp.
+// A counter update that publishes (release) everything this warp wrote before it (the
+// __syncwarp() before each call orders the other lanes' writes first).
 Q4_DEVINL void red_release_add(int *p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-Q4_DEVINL int atom_acq_rel_add(int *p, int v) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
 }
 Q4_DEVINL void tmap_acquire(const CUtensorMap *tm) {
     asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(tm) : "memory");
@@ -120,9 +130,8 @@ Q4_DEVINL void tma_load_2d_g(void *dst, const CUtensorMap *tmap, uint64_t *bar, 
         ::"r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
-
-// The CTA that owns tile u of a level with U tiles.
-Q4_DEVINL int cta_of(int64_t u, int64_t U, int G) { return (int)(((u + 1) * G - 1) / U); }
+Q4_DEVINL void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+Q4_DEVINL void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 // Entry of tile u (level-local), searching forward from e.
 Q4_DEVINL int locate(const StackEntry *ent, int e, int e_end, int64_t u) {
@@ -157,19 +166,50 @@ Q4_DEVINL bool wait_counter(const int *p, int target, uint64_t limit_ns) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
-        __nanosleep(64);
+        __nanosleep(32);
         if (ld_acquire(p) >= target) return true;
         if (global_ns() - t0 > limit_ns) return false;
     }
 }
 
+constexpr int kMaxUcap = 64;  // tiles whose slots are built at once, at most
+#ifndef Q4_STACK_MAX_READ_PARTS
+#define Q4_STACK_MAX_READ_PARTS 1000
+#endif
+// A level reads x as the parts of the previous level's GEMV when each row has at most this
+// many parts; with more, the reads cost more than waiting for the sums in y.
+constexpr int kMaxReadParts = Q4_STACK_MAX_READ_PARTS;
+
+// Warp-wide: every level j in [lo, hi] has all its sums of split row blocks in y (lane q
+// watches level lo + q).
+Q4_DEVINL bool wait_fin(const int *fin_done, const StackLevel *lev, int lo, int hi, uint64_t limit_ns, int lane) {
+    for (int j0 = lo; j0 <= hi; j0 += 32) {
+        const int j = j0 + lane;
+        const int target = j <= hi ? lev[j].fin_target : 0;
+        auto done = [&]() { return j > hi || ld_acquire(fin_done + j) >= target; };
+        if (__all_sync(0xffffffffu, done())) continue;
+        const uint64_t t0 = global_ns();
+        for (;;) {
+            __nanosleep(32);
+            if (__all_sync(0xffffffffu, done())) break;
+            if (__any_sync(0xffffffffu, global_ns() - t0 > limit_ns)) return false;
+        }
+    }
+    return true;
+}
+
+// First scale group of k-stage s.
+template <int GPS, int STAGEK>
+Q4_DEVINL int stage_group(int s, int group) {
+    return GPS > 0 ? s * GPS : (s * STAGEK) / group;
+}
+
 template <int BITS, int L, int GPS, bool XBF16>
 __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     constexpr int SPS = kTileBytes / (4 * L);
-    constexpr int KTI = BITS == 4 ? L / 2 : L / 4;
-    constexpr int KTS = SPS * KTI;
     constexpr int WPT = L / 4;
     constexpr int STAGEK = kTileBytes * 8 / BITS;
+    constexpr int LANES = STAGEK / 8;
     constexpr int GS = GPS > 0 ? GPS : 1;
     constexpr int FSLOT = slot1_bytes<BITS>();  // B fragments of one tile + format header
     extern __shared__ uint8_t smem_raw[];
@@ -179,6 +219,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     uint64_t *full = reinterpret_cast<uint64_t *>(bbuf + (size_t)a.ucap * FSLOT);
     uint64_t *empty = full + kRing;
     int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: a wait of this CTA gave up
+    int *finq = flag + 4;  // [warp][2][4] pending sums of split row blocks: {entry, rb, parts, level}
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, G = a.G;
@@ -223,6 +264,21 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 }
                 ++issued[slot];
                 if (++slot == kRing) { slot = 0; ++round; }
+                if (i == 0 || cu.s == 0) {
+                    // the scales of this CTA's stretch of the row block, into L2 ahead of use
+                    const int s_end = min(S - 1, cu.s + (n - i) - 1);
+                    const int g_lo = stage_group<GPS, STAGEK>(cu.s, E->group);
+                    const int g_hi = min(E->spr - 1, stage_group<GPS, STAGEK>(s_end, E->group) + GS - 1);
+                    const int N = E->N, spr = E->spr;
+                    const float *sc = E->scales;
+                    for (int rr = lane; rr < kSRows; rr += 32) {
+                        const int row = cu.rb * kSRows + rr;
+                        if (row >= N) break;
+                        const uintptr_t lo = (uintptr_t)(sc + (size_t)row * spr + g_lo) & ~(uintptr_t)127;
+                        const uintptr_t hi = (uintptr_t)(sc + (size_t)row * spr + g_hi);
+                        for (uintptr_t q = lo; q <= hi; q += 128) prefetch_l2(reinterpret_cast<const void *>(q));
+                    }
+                }
             }
         }
         // drain: every copy issued into this CTA's shared memory has landed before it exits
@@ -242,17 +298,91 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
         }
         float ys0 = 0.f, ys1 = 0.f;  // this lane's share of rows pr and pr + 8
         int slot = 0, round = 0;
-        for (int l = 0; l < a.L; ++l) {
-            const StackLevel lv = a.lev[l];
-            const int *us = a.ustart + (size_t)l * (G + 1);
-            const int64_t u0 = us[c];
-            const int n = us[c + 1] - us[c];
-            if (n == 0) continue;
+        // split row blocks whose last part this CTA holds, by level parity: their sums (rows
+        // of y) are written at the start of the level after next (see the file comment)
+        int *fq = finq + warp * 8;
+        if (lane == 0) fq[0] = fq[4] = -1;
+        __syncwarp();
+        // the sum of split row block f, parts in order, by warps w0..14 (the others are busy
+        // building); one release for the block once all of them have written their rows
+        auto finalize = [&](const int *f, int w0) {
+            if (warp < w0) return;
+            const int nw = kConsumers - w0;
+            const StackEntry *fe = a.ent + f[0];
+            const int np = f[2];
+            const size_t st = (size_t)fe->npad;
+            for (int rr = (warp - w0) * 32 + lane; rr < kSRows; rr += nw * 32) {
+                const int row = f[1] * kSRows + rr;
+                if (row < fe->N) {
+                    const float *pp = fe->parts + row;
+                    float v = __ldcg(pp);
+                    for (int q = 1; q < np; ++q) v += __ldcg(pp + q * st);
+                    if (np < fe->pmax) v += 0.f;  // as the sum over all pmax parts, zeros included
+                    fe->y[row] = v;
+                }
+            }
+            named_barrier_sync(2, nw * 32);
+            if (warp == w0 && lane == 0) {
+                __threadfence();
+                red_release_add(a.fin_done + f[3], 1);
+            }
+        };
+        for (int l = 0; l <= a.L; ++l) {
+            int64_t u0 = 0;
+            int n = 0, pcur = 0;
+            if (l < a.L) {
+                const int *us = a.ustart + (size_t)l * (G + 1);
+                u0 = us[c];
+                n = us[c + 1] - us[c];
+                pcur = a.pfirst[(size_t)l * G + c];
+            }
+            int *f_old = fq + 4 * (l & 1);        // a block of level l - 2
+            int *f_new = fq + 4 * ((l + 1) & 1);  // a block of level l - 1
+            const bool has_old = f_old[0] >= 0, has_new = f_new[0] >= 0;
+            if (n == 0 && !has_old && !has_new) continue;
+            StackLevel lv;
+            Cursor cu;
+            if (l < a.L) lv = a.lev[l];
+            if (n > 0) {
+                cu = cursor_at(a.ent, lv, u0);
+                // the first tile's scale lines, into L1 while this level waits
+                const StackEntry *E0 = a.ent + cu.e;
+                const int gb = stage_group<GPS, STAGEK>(cu.s, E0->group);
+                const int N0 = E0->N;
+                prefetch_l1(E0->scales + (size_t)min(cu.rb * kSRows + pr, N0 - 1) * E0->spr + gb);
+                prefetch_l1(E0->scales + (size_t)min(cu.rb * kSRows + pr + 8, N0 - 1) * E0->spr + gb);
+            }
             if (l > 0) {
-                // the activations of this level are complete once every warp of every row
-                // block of the previous level has published its rows
-                if (ct == 0 && !timed_out)
-                    timed_out = !wait_counter(a.level_done + (l - 1), kConsumers * a.lev[l - 1].T, a.wait_ns);
+                // the activations are complete once every warp of every part of the previous
+                // level has published its rows, and the levels this one needs have their sums
+                if (warp == 0 && !timed_out) {
+                    bool ok = true;
+                    if (lane == 0) ok = wait_counter(a.parts_done + (l - 1), a.lev[l - 1].parts_target, a.wait_ns);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok && l < a.L) ok = wait_fin(a.fin_done, a.lev, lv.fin_lo, lv.fin_hi, a.wait_ns, lane);
+                    timed_out = !ok;
+                }
+                named_barrier_sync(1, kConsumerThreads);
+            }
+            // pending sums: level l - 2's blocks (their parts were complete before level l - 1
+            // started) and level l - 1's (complete now), the latter only when this level reads
+            // their y, or has no tiles, or is the end. Warps with no slot to build do them
+            // while the others build.
+            const bool now_new = has_new && (l == a.L || n == 0 || lv.needs_final);
+            const int w_free = (l == a.L || n == 0 || lv.needs_final) ? 0 : min(kConsumers, min(n, a.ucap));
+            if (w_free < kConsumers) {
+                if (has_old) finalize(f_old, w_free);
+                if (now_new) finalize(f_new, w_free);
+            }
+            if (lane == 0) {
+                if (has_old && w_free < kConsumers) f_old[0] = -1;
+                if (now_new) f_new[0] = -1;
+            }
+            __syncwarp();
+            if (l == a.L || n == 0) continue;
+            if (lv.needs_final) {
+                named_barrier_sync(1, kConsumerThreads);
+                if (warp == 0 && !timed_out) timed_out = !wait_fin(a.fin_done, a.lev, l - 1, l - 1, a.wait_ns, lane);
                 named_barrier_sync(1, kConsumerThreads);
             }
             // B fragments of tiles [i0, i1) of this level (i relative to u0), one tile per warp
@@ -261,32 +391,65 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 for (int i = i0 + warp; i < i1; i += kConsumers) {
                     const Cursor bc = cursor_at(a.ent, lv, u0 + i);
                     const StackEntry *BE = a.ent + bc.e;
-                    build_slot1<BITS, L, XBF16, true>(bbuf + (size_t)(i - i0) * FSLOT, BE->x, bc.s * STAGEK, BE->K,
-                                                     a.P, lane);
+                    uint8_t *bs = bbuf + (size_t)(i - i0) * FSLOT;
+                    const float *xp = XBF16 ? nullptr : BE->xparts;
+                    if (!xp) {
+                        build_slot1<BITS, L, XBF16, true>(bs, BE->x, bc.s * STAGEK, BE->K, a.P, lane);
+                        continue;
+                    }
+                    // x = the sum of the producing GEMV's parts of these rows, in part order
+                    float v[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[q] = 0.f;
+                    const int k = bc.s * STAGEK + 8 * lane;
+                    if (lane < LANES && k < BE->K) {
+                        const float4 *src = reinterpret_cast<const float4 *>(xp + k);
+                        const size_t st4 = (size_t)BE->xstride / 4;
+                        const int pm = BE->xpmax;
+                        float4 s0 = __ldcg(src), s1 = __ldcg(src + 1);
+                        for (int q0 = 1; q0 < pm; q0 += 2) {
+                            const bool two = q0 + 1 < pm;
+                            const float4 b0 = __ldcg(src + q0 * st4), b1 = __ldcg(src + q0 * st4 + 1);
+                            float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+                            if (two) {
+                                c0 = __ldcg(src + (q0 + 1) * st4);
+                                c1 = __ldcg(src + (q0 + 1) * st4 + 1);
+                            }
+                            s0.x += b0.x; s0.y += b0.y; s0.z += b0.z; s0.w += b0.w;
+                            s1.x += b1.x; s1.y += b1.y; s1.z += b1.z; s1.w += b1.w;
+                            if (two) {
+                                s0.x += c0.x; s0.y += c0.y; s0.z += c0.z; s0.w += c0.w;
+                                s1.x += c1.x; s1.y += c1.y; s1.z += c1.z; s1.w += c1.w;
+                            }
+                        }
+                        v[0] = s0.x; v[1] = s0.y; v[2] = s0.z; v[3] = s0.w;
+                        v[4] = s1.x; v[5] = s1.y; v[6] = s1.z; v[7] = s1.w;
+                    }
+                    build_slot1_v<BITS, L>(bs, v, a.P, lane);
                 }
             };
             int chunk_lo = 0, chunk_hi = min(n, a.ucap);
             build(0, chunk_hi);
+            if (has_old && w_free == kConsumers) {  // every warp built: the sum comes after
+                finalize(f_old, 0);
+                if (lane == 0) f_old[0] = -1;
+                __syncwarp();
+            }
             named_barrier_sync(1, kConsumerThreads);
 
-            Cursor cu = cursor_at(a.ent, lv, u0);
             const StackEntry *E = a.ent + cu.e;
-            int S = E->S, R = E->R, N = E->N, K = E->K, task_base = E->task_base, spr = E->spr, group = E->group;
-            float *y = E->y;
+            int S = E->S, R = E->R, N = E->N, K = E->K, spr = E->spr, group = E->group;
             const float *scales = E->scales;
-            int64_t unit_base = E->unit_base;
-            int seg_s0 = cu.s;  // first stage of the current row block in this CTA
+            int pend = 0;  // parts written and not yet published
             for (int i = 0; i < n; ++i) {
                 if (i > 0) {
                     if (cursor_next(cu, S, R)) {
                         E = a.ent + cu.e;
-                        S = E->S; R = E->R; N = E->N; K = E->K; task_base = E->task_base;
+                        S = E->S; R = E->R; N = E->N; K = E->K;
                         spr = E->spr; group = E->group;
-                        y = E->y;
                         scales = E->scales;
-                        unit_base = E->unit_base;
                     }
-                    if (cu.s == 0) seg_s0 = 0;
+                    if (cu.s == 0) pcur = 0;  // a row block that starts in this CTA's range
                 }
                 if (i == chunk_hi) {
                     named_barrier_sync(1, kConsumerThreads);  // every warp is done with the last chunk
@@ -302,7 +465,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 // their latency overlaps the wait for the tile
                 float s0r[GS], s1r[GS];
                 {
-                    const int gbase = GPS > 0 ? cu.s * GPS : (cu.s * STAGEK) / group;
+                    const int gbase = stage_group<GPS, STAGEK>(cu.s, group);
                     const int ng = min(GS, spr - gbase);
                     const float *sp0 = scales + (size_t)min(cu.rb * kSRows + pr, N - 1) * spr + gbase;
                     const float *sp1 = scales + (size_t)min(cu.rb * kSRows + pr + 8, N - 1) * spr + gbase;
@@ -338,10 +501,9 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                         stage1_pieces<BITS, L, GPS, false>(A0, A1, slt, lane, s0r, s1r, nsl, ys0, ys1);
                 }
 
-                // ---- end of this CTA's share of row block rb: each warp finishes its 16 rows ----
-                if (cu.s == S - 1 || i == n - 1) {
-                    const int T = task_base + cu.rb;
-                    const bool whole = cu.s == S - 1 && seg_s0 == 0;
+                // ---- end of this CTA's part of row block rb: each warp publishes its 16 rows ----
+                const bool block_end = cu.s == S - 1 || i == n - 1;
+                if (block_end) {
                     // rows pr and pr + 8: the four lanes of each row add their shares
                     float r0 = ys0 + __shfl_xor_sync(0xffffffffu, ys0, 1);
                     float r1 = ys1 + __shfl_xor_sync(0xffffffffu, ys1, 1);
@@ -353,69 +515,33 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                     const float v = (t & 1) ? r1 : r0;
                     const bool writer = t < 2;
                     const int nrow = cu.rb * kSRows + r;
-                    if (whole) {
-                        if (writer && nrow < N) y[nrow] = v;
-                        __syncwarp();
-                        if (lane == 0) red_release_add(a.level_done + l, 1);
-                    } else {
-                        // the partial sums of a CTA's rows go to its slot 0 when the row block
-                        // starts inside the CTA's range, else to slot 1 (a range holds parts of
-                        // at most two split row blocks)
-                        const int64_t tf = unit_base + (int64_t)cu.rb * S;
-                        if (writer) a.partial[((size_t)c * 2 + (u0 >= tf ? 0 : 1)) * kSRows + r] = v;
-                        __syncwarp();
-                        // the CTAs holding parts of this row block (lanes take one each), and
-                        // whether this warp is the last of them to arrive for its rows
-                        const int cf = cta_of(tf, lv.U, G), clast = cta_of(tf + S - 1, lv.U, G);
-                        int arrivals = 0;
-                        for (int base = cf; base <= clast; base += 32) {
-                            const int cc = base + lane;
-                            const bool in = cc <= clast && us[cc] < us[cc + 1];
-                            arrivals += __popc(__ballot_sync(0xffffffffu, in));
-                        }
-                        int last = 0;
-                        if (lane == 0)
-                            last = atom_acq_rel_add(a.task_cnt + (size_t)T * kConsumers + warp, 1) == arrivals - 1;
-                        last = __shfl_sync(0xffffffffu, last, 0);
-                        if (last) {
-                            // lane j reads the 16 partial sums of CTA cf + j; the warp adds them
-                            // in a fixed tree order (deterministic), 32 CTAs at a time in order;
-                            // lane rr keeps row 16 * warp + rr
-                            __syncwarp();
-                            float mine = 0.f;
-                            for (int base = cf; base <= clast; base += 32) {
-                                const int cc = base + lane;
-                                const bool in = cc <= clast && us[cc] < us[cc + 1];
-                                float pv[16];
-                                if (in) {
-                                    const float4 *src = reinterpret_cast<const float4 *>(
-                                        a.partial + ((size_t)cc * 2 + (us[cc] >= tf ? 0 : 1)) * kSRows + 16 * warp);
-#pragma unroll
-                                    for (int q = 0; q < 4; ++q) {
-                                        const float4 f4 = __ldcg(src + q);
-                                        pv[4 * q] = f4.x; pv[4 * q + 1] = f4.y; pv[4 * q + 2] = f4.z; pv[4 * q + 3] = f4.w;
-                                    }
-                                } else {
-#pragma unroll
-                                    for (int q = 0; q < 16; ++q) pv[q] = 0.f;
-                                }
-#pragma unroll
-                                for (int rr = 0; rr < 16; ++rr) {
-                                    float t2 = pv[rr];
-#pragma unroll
-                                    for (int m = 16; m >= 1; m >>= 1) t2 += __shfl_xor_sync(0xffffffffu, t2, m);
-                                    if (lane == rr) mine = base == cf ? t2 : mine + t2;
-                                }
-                            }
-                            const int nr = cu.rb * kSRows + 16 * warp + lane;
-                            if (lane < 16 && nr < N) y[nr] = mine;
-                            __syncwarp();
-                            if (lane == 0) {
-                                a.task_cnt[(size_t)T * kConsumers + warp] = 0;
-                                red_release_add(a.level_done + l, 1);
-                            }
+                    const bool last_part = cu.s == S - 1;  // the row block ends in this CTA's range
+                    const bool src = E->is_src != 0;
+                    if (writer && nrow < N) {
+                        if (last_part && pcur == 0) E->y[nrow] = v;  // the whole row block: v is y
+                        if (pcur > 0 || !last_part || src) {
+                            float *pp = E->parts + nrow;
+                            const size_t st = (size_t)E->npad;
+                            pp[pcur * st] = v;
+                            if (last_part && src)
+                                for (int q = pcur + 1; q < E->pmax; ++q) pp[q * st] = 0.f;
                         }
                     }
+                    ++pend;
+                    if (last_part && pcur > 0 && lane == 0) {
+                        int *f = fq + 4 * (l & 1);  // summed at the start of level l + 2
+                        f[0] = cu.e;
+                        f[1] = cu.rb;
+                        f[2] = pcur + 1;
+                        f[3] = l;
+                    }
+                }
+                // parts are published one tile late (their stores have landed by then, so the
+                // release does not stall), and at once at the end of the CTA's range
+                if (pend > 0 && (!block_end || i == n - 1)) {
+                    __syncwarp();
+                    if (lane == 0) red_release_add(a.parts_done + l, pend);
+                    pend = 0;
                 }
             }
         }
@@ -423,19 +549,15 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     if (timed_out) flag[0] = 1;
     __syncthreads();
     if (threadIdx.x == 0) {
-        if (flag[0]) {
-            if (a.status) atomicOr(a.status, Q4_STATUS_TIMEOUT);
-            atomicExch(a.tflag, 1);
-        }
+        if (flag[0] && a.status) atomicOr(a.status, Q4_STATUS_TIMEOUT);
         __threadfence();
         const int old = atomicAdd(a.finished, 1);
         if (old == G - 1) {
             // every CTA is done with the counters: return them to zero for the next launch
             __threadfence();
-            for (int l = 0; l < a.L; ++l) a.level_done[l] = 0;
-            if (atomicAdd(a.tflag, 0)) {
-                for (int i = 0; i < a.n_tasks * kConsumers; ++i) a.task_cnt[i] = 0;
-                *a.tflag = 0;
+            for (int l = 0; l < a.L; ++l) {
+                a.parts_done[l] = 0;
+                a.fin_done[l] = 0;
             }
             *a.finished = 0;
             __threadfence();
@@ -452,8 +574,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
 namespace q4 {
 namespace {
 
-constexpr int kPlanGrid = 148 * kCtasPerSm;  // partial-sum slots are sized for a full B200
-constexpr uint64_t kPlanMagic = 0x71347374616b3031ull;
+constexpr int kPlanGrid = 148 * kCtasPerSm;  // the workspace is sized for a full B200
+constexpr uint64_t kPlanMagic = 0x71347374616b3032ull;
 
 inline size_t al256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -474,14 +596,26 @@ bool stack_format(int bits, int64_t K, int64_t group, int *L, int *gps) {
     return true;
 }
 
+inline int64_t stages_of(int64_t K, int bits) { return (K * bits / 8 + kTileBytes - 1) / kTileBytes; }
+inline int64_t blocks_of(int64_t N) { return (N + kSRows - 1) / kSRows; }
+inline int64_t npad_of(int64_t N) { return (N + 3) / 4 * 4; }
+
+// At most how many CTA ranges a row block of S tiles meets when a level of U tiles is
+// split over G CTAs: ranges are at least max(1, U / G) tiles long. The bound only falls
+// as G falls, so the workspace sized with the largest grid serves every smaller one.
+inline int64_t parts_bound(int64_t S, int64_t U, int64_t G) {
+    const int64_t m = std::max<int64_t>(1, U / G);
+    return std::min<int64_t>(S, 1 + (S - 1 + m - 1) / m);
+}
+
 struct StackLayout {
-    int L, gps, nlev, n_tasks;
-    size_t off_ent, off_lev, off_cnt, off_done, off_misc, off_part, off_us, bytes;
+    int L, gps, nlev;
+    size_t part_floats;  // floats of one parts buffer (three rotate over the levels)
+    size_t off_ent, off_lev, off_cnt, off_part, off_us, off_pf, bytes;
 };
 
 q4_status stack_layout(const q4_stack_gemv *gv, int32_t count, int bits, q4_xdtype xt, StackLayout *lo) {
     if (!gv || count < 1 || (bits != 4 && bits != 8) || (xt != Q4_X_F32 && xt != Q4_X_BF16)) return Q4_ERR_ARG;
-    int64_t tasks = 0;
     for (int32_t i = 0; i < count; ++i) {
         const q4_stack_gemv &g = gv[i];
         if (!g.payload || !g.scales || !g.x || !g.y) return Q4_ERR_ARG;
@@ -497,19 +631,29 @@ q4_status stack_layout(const q4_stack_gemv *gv, int32_t count, int bits, q4_xdty
         } else if (L != lo->L || gps != lo->gps) {
             return Q4_ERR_UNSUPPORTED;  // one kernel variant per stack
         }
-        tasks += (g.N + kSRows - 1) / kSRows;
     }
-    if (tasks > (int64_t)1 << 30) return Q4_ERR_UNSUPPORTED;
     lo->nlev = gv[count - 1].level + 1;
-    lo->n_tasks = (int)tasks;
+    // the largest parts buffer any level needs on any grid up to a full B200
+    size_t pmax_floats = 0;
+    for (int32_t i = 0; i < count;) {
+        int32_t j = i;
+        int64_t U = 0;
+        for (; j < count && gv[j].level == gv[i].level; ++j) U += blocks_of(gv[j].N) * stages_of(gv[j].K, bits);
+        if (U >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
+        size_t f = 0;
+        for (int32_t e = i; e < j; ++e)
+            f += (size_t)parts_bound(stages_of(gv[e].K, bits), U, kPlanGrid) * (size_t)npad_of(gv[e].N);
+        pmax_floats = std::max(pmax_floats, f);
+        i = j;
+    }
+    lo->part_floats = pmax_floats;
     lo->off_ent = 0;
     lo->off_lev = al256((size_t)count * sizeof(StackEntry));
-    lo->off_cnt = lo->off_lev + al256((size_t)lo->nlev * sizeof(StackLevel));
-    lo->off_done = lo->off_cnt + al256((size_t)lo->n_tasks * kConsumers * 4);
-    lo->off_misc = lo->off_done + al256((size_t)lo->nlev * 4);
-    lo->off_part = lo->off_misc + 256;
-    lo->off_us = lo->off_part + al256((size_t)kPlanGrid * 2 * kSRows * 4);
-    lo->bytes = lo->off_us + al256((size_t)lo->nlev * (kPlanGrid + 1) * 4);
+    lo->off_cnt = lo->off_lev + al256((size_t)lo->nlev * sizeof(StackLevel));       // parts_done, fin_done, finished
+    lo->off_part = lo->off_cnt + al256((size_t)(2 * lo->nlev + 1) * 4);
+    lo->off_us = lo->off_part + 3 * al256(pmax_floats * 4);
+    lo->off_pf = lo->off_us + al256((size_t)lo->nlev * (kPlanGrid + 1) * 4);
+    lo->bytes = lo->off_pf + al256((size_t)lo->nlev * kPlanGrid * 4);
     return Q4_OK;
 }
 
@@ -569,47 +713,12 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     StackKernel kern = stack_kernel(bits, lo.L, lo.gps, bf16);
     if (!kern) return Q4_ERR_UNSUPPORTED;
 
-    // tables
-    std::vector<StackEntry> ent(count);
-    std::vector<StackLevel> lev(lo.nlev);
-    int task_base = 0;
-    for (int l = 0, i = 0; l < lo.nlev; ++l) {
-        StackLevel &lv = lev[l];
-        lv.e0 = i;
-        lv.U = 0;
-        lv.T = 0;
-        lv.pad = 0;
-        for (; i < count && gemvs[i].level == l; ++i) {
-            const q4_stack_gemv &g = gemvs[i];
-            StackEntry &E = ent[i];
-            std::memset(&E, 0, sizeof E);
-            if (!encode_payload_map(&E.tm, g.payload, g.N, g.K, bits, kSRows)) return Q4_ERR_UNSUPPORTED;
-            E.scales = g.scales;
-            E.x = g.x;
-            E.y = g.y;
-            E.N = (int)g.N;
-            E.K = (int)g.K;
-            E.group = (int)g.group;
-            E.spr = (int)(g.K / g.group);
-            E.S = (int)((g.K * bits / 8 + kTileBytes - 1) / kTileBytes);
-            E.R = (int)((g.N + kSRows - 1) / kSRows);
-            E.task_base = task_base;
-            E.level = l;
-            E.unit_base = lv.U;
-            lv.U += (int64_t)E.R * E.S;
-            lv.T += E.R;
-            task_base += E.R;
-        }
-        lv.ne = i - lv.e0;
-    }
-
-    // shared memory and grid
+    // grid and shared memory
     const size_t fslot = bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>();  // B fragments + header of a tile
-    const int gsl = lo.gps > 0 ? lo.gps : 1;
-    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16;
+    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4;
     if (fixed + fslot > (size_t)kSmemBudget) return Q4_ERR_UNSUPPORTED;
     int ucap = (int)((kSmemBudget - fixed) / fslot);
-    if (ucap > 64) ucap = 64;
+    if (ucap > kMaxUcap) ucap = kMaxUcap;
     const size_t smem = fixed + (size_t)ucap * fslot;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_error(e, "stack kernel attribute");
@@ -623,20 +732,122 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     int grid = sms * (per_sm < kCtasPerSm ? per_sm : kCtasPerSm);
     if (grid > kPlanGrid) grid = kPlanGrid;
 
-    // each CTA's first tile in each level: an even split of the level's tiles
+    char *w = static_cast<char *>(workspace);
+    float *parts_buf[3];
+    for (int q = 0; q < 3; ++q) parts_buf[q] = reinterpret_cast<float *>(w + lo.off_part + q * al256(lo.part_floats * 4));
+    std::vector<StackEntry> ent(count);
+    std::vector<StackLevel> lev(lo.nlev);
     std::vector<int> ustart((size_t)lo.nlev * (grid + 1));
+    std::vector<int> pfirst((size_t)lo.nlev * grid, 0);
+    for (int l = 0, i = 0; l < lo.nlev; ++l) {
+        StackLevel &lv = lev[l];
+        std::memset(&lv, 0, sizeof lv);
+        lv.e0 = i;
+        for (; i < count && gemvs[i].level == l; ++i) {
+            const q4_stack_gemv &g = gemvs[i];
+            StackEntry &E = ent[i];
+            std::memset(&E, 0, sizeof E);
+            if (!encode_payload_map(&E.tm, g.payload, g.N, g.K, bits, kSRows)) return Q4_ERR_UNSUPPORTED;
+            E.scales = g.scales;
+            E.x = g.x;
+            E.y = g.y;
+            E.N = (int)g.N;
+            E.K = (int)g.K;
+            E.group = (int)g.group;
+            E.spr = (int)(g.K / g.group);
+            E.S = (int)stages_of(g.K, bits);
+            E.R = (int)blocks_of(g.N);
+            E.npad = (int)npad_of(g.N);
+            E.level = l;
+            E.unit_base = lv.U;
+            lv.U += (int64_t)E.R * E.S;
+        }
+        lv.ne = i - lv.e0;
+        // each CTA's first tile: an even split of the level's tiles, every range non-empty
+        // when there are at least as many tiles as CTAs (else one tile for each of the first U)
+        int *us = ustart.data() + (size_t)l * (grid + 1);
+        for (int cc = 0; cc <= grid; ++cc)
+            us[cc] = lv.U < grid ? (int)std::min<int64_t>(cc, lv.U) : (int)(lv.U * cc / grid);
+        auto cta_of = [&](int64_t u) {  // the CTA whose range holds tile u
+            return (int)(std::upper_bound(us, us + grid + 1, (int)u) - us) - 1;
+        };
+        // parts of every row block; this level's parts buffer (by level parity)
+        size_t off = 0;
+        int64_t pairs = 0, split = 0;
+        for (int ei = lv.e0; ei < lv.e0 + lv.ne; ++ei) {
+            StackEntry &E = ent[ei];
+            int pm = 1;
+            for (int rb = 0; rb < E.R; ++rb) {
+                const int64_t tf = E.unit_base + (int64_t)rb * E.S;
+                const int np = cta_of(tf + E.S - 1) - cta_of(tf) + 1;
+                pm = std::max(pm, np);
+                pairs += np;
+                split += np > 1;
+            }
+            E.pmax = pm;
+            E.parts = parts_buf[l % 3] + off;
+            off += (size_t)pm * E.npad;
+        }
+        if (off > lo.part_floats) return Q4_ERR_WORKSPACE;  // cannot happen with grid <= kPlanGrid
+        if (pairs * kConsumers >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
+        lv.parts_target = (int)(pairs * kConsumers);
+        lv.fin_target = (int)split;
+        for (int cc = 0; cc < grid; ++cc) {
+            if (us[cc] == us[cc + 1]) continue;
+            int ei = lv.e0;
+            while (ei + 1 < lv.e0 + lv.ne && us[cc] >= ent[ei + 1].unit_base) ++ei;
+            const int64_t tf = ent[ei].unit_base + (us[cc] - ent[ei].unit_base) / ent[ei].S * ent[ei].S;
+            pfirst[(size_t)l * grid + cc] = cc - cta_of(tf);
+        }
+    }
+    // x of level l read as the parts of a level l - 1 GEMV whose y holds it (fp32, 16-byte
+    // aligned slice). x overlapping the y of level l - 1 any other way: that level writes
+    // its sums at the next start and level l waits for them; overlapping the y of an older
+    // level: level l waits for that level's sums. Every level waits for the sums of three
+    // levels back (the parts buffers rotate over three levels).
     for (int l = 0; l < lo.nlev; ++l) {
-        if (lev[l].U >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
-        for (int cc = 0; cc <= grid; ++cc) ustart[(size_t)l * (grid + 1) + cc] = (int)(lev[l].U * cc / grid);
+        lev[l].fin_lo = l >= 3 ? l - 3 : 0;
+        lev[l].fin_hi = l >= 3 ? l - 3 : -1;
+    }
+    for (int i = 0; i < count; ++i) {
+        StackEntry &E = ent[i];
+        const int l = E.level;
+        const uintptr_t x0 = (uintptr_t)E.x;
+        const uintptr_t x1 = x0 + (uintptr_t)E.K * (bf16 ? 2 : 4);
+        for (int j = 0; j < lev[l].e0; ++j) {
+            StackEntry &P = ent[j];
+            const uintptr_t y0 = (uintptr_t)P.y, y1 = y0 + (uintptr_t)P.N * 4;
+            if (x1 <= y0 || x0 >= y1) continue;
+            if (P.level == l - 1) {
+                if (!bf16 && !E.xparts && x0 >= y0 && x1 <= y1 && (x0 - y0) % 16 == 0 && P.pmax <= kMaxReadParts) {
+                    E.xparts = P.parts + (x0 - y0) / 4;
+                    E.xpmax = P.pmax;
+                    E.xstride = P.npad;
+                    P.is_src = 1;
+                } else {
+                    lev[l].needs_final = 1;
+                    lev[l - 1].fin_early = 1;
+                }
+            } else {
+                StackLevel &lv = lev[l];
+                if (lv.fin_hi < lv.fin_lo) {
+                    lv.fin_lo = lv.fin_hi = P.level;
+                } else {
+                    lv.fin_lo = std::min(lv.fin_lo, P.level);
+                    lv.fin_hi = std::max(lv.fin_hi, P.level);
+                }
+            }
+        }
     }
     // copy the tables, zero the counters; the host tables can go once the stream is done
-    char *w = static_cast<char *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((e = cudaMemcpyAsync(w + lo.off_ent, ent.data(), ent.size() * sizeof(StackEntry), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(w + lo.off_lev, lev.data(), lev.size() * sizeof(StackLevel), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(w + lo.off_us, ustart.data(), ustart.size() * sizeof(int), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(w + lo.off_pf, pfirst.data(), pfirst.size() * sizeof(int), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
         (e = cudaMemsetAsync(w + lo.off_cnt, 0, lo.off_part - lo.off_cnt, s)) != cudaSuccess ||
         (e = cudaStreamSynchronize(s)) != cudaSuccess)
@@ -647,19 +858,16 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     p.kern = kern;
     p.args.ent = reinterpret_cast<const StackEntry *>(w + lo.off_ent);
     p.args.lev = reinterpret_cast<const StackLevel *>(w + lo.off_lev);
-    p.args.task_cnt = reinterpret_cast<int *>(w + lo.off_cnt);
-    p.args.level_done = reinterpret_cast<int *>(w + lo.off_done);
-    p.args.finished = reinterpret_cast<int *>(w + lo.off_misc);
-    p.args.tflag = reinterpret_cast<int *>(w + lo.off_misc) + 1;
-    p.args.partial = reinterpret_cast<float *>(w + lo.off_part);
+    p.args.parts_done = reinterpret_cast<int *>(w + lo.off_cnt);
+    p.args.fin_done = p.args.parts_done + lo.nlev;
+    p.args.finished = p.args.fin_done + lo.nlev;
     p.args.ustart = reinterpret_cast<const int *>(w + lo.off_us);
+    p.args.pfirst = reinterpret_cast<const int *>(w + lo.off_pf);
     p.args.status = nullptr;
     p.args.G = grid;
     p.args.L = lo.nlev;
-    p.args.n_tasks = lo.n_tasks;
     p.args.P = bf16 ? 1 : 3;
     p.args.ucap = ucap;
-    p.args.gs = gsl;
     p.args.wait_ns = kWaitLimitNs;
     p.grid = grid;
     p.smem = smem;

@@ -264,3 +264,49 @@ def test_stages_of_every_activation_range(q4, bits):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     check_all(gemvs, [("w", 0, N, K, 128, p, s), ("w2", 0, N, N, 128, p2, s2)], bits, f"ranges int{bits}")
+
+
+def test_x_read_as_slices_of_earlier_outputs(q4):
+    # every way a level can read earlier outputs: a slice of one previous-level y at a
+    # 16-byte offset from its start (read through that GEMV's parts), a slice at another
+    # offset and a slice across two GEMVs' y (both read from y once the sums are written),
+    # and outputs of two levels back. The levels are small (fewer tiles than CTAs), so
+    # every row block is split into parts.
+    import torch
+
+    rng = np.random.default_rng(31)
+    h = torch.from_numpy(rng.normal(0, 1, 1024).astype(np.float32)).cuda()
+    Y = torch.zeros(1701, dtype=torch.float32, device="cuda")  # y of A, one unused float, y of B
+    yC = torch.empty(300, dtype=torch.float32, device="cuda")
+    spec = [  # name, N, K, level, x
+        ("A", 1000, 1024, 0, h), ("B", 700, 1024, 0, h),
+        ("C", 300, 512, 1, Y[8:520]),        # A's rows 8..519: through A's parts
+        ("D", 64, 256, 1, Y[1004:1260]),     # B's rows 3..258: B's y is not 16-byte aligned
+        ("E", 130, 256, 1, Y[992:1248]),     # across A, the unused float and B
+        ("F", 200, 512, 2, Y[0:512]),        # two levels back
+        ("G", 96, 256, 2, yC[0:256]),        # C's rows 0..255: through C's parts
+    ]
+    outs = {"A": Y[:1000], "B": Y[1001:], "C": yC}
+    gemvs, host = [], []
+    for name, N, K, lvl, x in spec:
+        assert x.data_ptr() % 16 == 0
+        w = rng.normal(0, 1.0 / np.sqrt(K), (N, K)).astype(np.float32)
+        p, s, _ = oracle.pack(w, 4, 128)
+        y = outs.get(name)
+        if y is None:
+            y = torch.empty(N, dtype=torch.float32, device="cuda")
+        gemvs.append(q4.StackGemv(torch.from_numpy(p).cuda(), torch.from_numpy(s).cuda(), x, y, N, K, 128, lvl))
+        host.append((name, lvl, N, K, 128, p, s))
+    # an x that does not start on a 16-byte boundary is rejected up front
+    bad = list(gemvs)
+    bad[3] = q4.StackGemv(bad[3].payload, bad[3].scales, Y[1005:1261], bad[3].y, 64, 256, 128, 1)
+    with pytest.raises(q4.Q4Error):
+        q4.DecodeStack(bad, 4)
+    st = q4.DecodeStack(gemvs, 4)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        st.run(status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert float(Y[1000]) == 0.0  # nobody writes between the two outputs
+    check_all(gemvs, host, 4, "slices")
