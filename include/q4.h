@@ -239,9 +239,12 @@ Q4_API q4_status qgemm_noalloc(const void *x, q4_xdtype xt, int64_t M, const uin
  *
  * GEMVs are grouped in levels: the GEMVs of level l may read (as x) what GEMVs of
  * levels < l write (as y), and nothing that GEMVs of level >= l write. Inside one
- * launch, level l starts reading x only once every GEMV of level l - 1 has written
- * all of y; weights stream continuously across levels. A transformer layer is four
- * levels: q|k|v, o, gate|up, down.
+ * launch, level l starts reading x only once every GEMV of level l - 1 has computed
+ * all of y: where x is a 16-byte aligned slice of one level l - 1 GEMV's y, it is read
+ * as the sum of the partial sums the kernel keeps for those rows (the very values that
+ * GEMV's y receives); any other x is read from memory once the y it overlaps is
+ * written. Weights stream continuously across levels. A transformer layer is four
+ * levels: q|k|v, o, gate|up, down. Every y is complete when the run ends.
  */
 typedef struct q4_stack_gemv {
     const uint8_t *payload;  /* [N][K*bits/8] from qpack of an [N][K] matrix, 16-byte aligned */
@@ -261,9 +264,10 @@ typedef struct q4_stack_plan {
 } q4_stack_plan;
 
 /* Workspace bytes q4_stack_prepare needs for these GEMVs: the GEMV and level tables
- * (one 2D TMA descriptor per GEMV), one counter per 128-row block and per level, and
- * the partial sums of row blocks split between CTAs (296 x 128 floats x 2). Returns 0
- * for arguments q4_stack_prepare rejects. */
+ * (one 2D TMA descriptor per GEMV), two counters per level, each CTA's share of every
+ * level, and three buffers for the partial sums of 240-row blocks split between CTAs
+ * (each sized for the level that needs most on a 148-SM B200). Returns 0 for
+ * arguments q4_stack_prepare rejects. */
 Q4_API size_t q4_stack_workspace_bytes(const q4_stack_gemv *gemvs, int32_t count, int bits, q4_xdtype xt);
 
 /*
