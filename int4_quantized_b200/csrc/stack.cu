@@ -89,7 +89,7 @@ struct alignas(64) StackEntry {
 struct StackLevel {
     int64_t U;             // tiles in the level
     int e0, ne;            // its GEMVs
-    int parts_target;      // arrivals that complete the level: 15 per (row block, part)
+    int parts_target;      // parts that complete the level (one arrival per part)
     int fin_target;        // arrivals that complete its sums of split row blocks: one per block
     int fin_lo, fin_hi;    // levels whose sums must be in y before this level starts (none: lo > hi)
     int needs_final;       // it reads a y of the previous level other than as a slice of parts
@@ -99,7 +99,7 @@ struct StackLevel {
 struct StackArgs {
     const StackEntry *ent;
     const StackLevel *lev;
-    int *parts_done;       // [L] published (row block, part, warp) triples per level
+    int *parts_done;       // [L] published (row block, part) pairs per level
     int *fin_done;         // [L] finished (split row block, warp) sums per level
     int *finished;         // CTAs done with the launch
     const int *ustart;     // [L][G + 1] first tile of each CTA's range in each level
@@ -120,6 +120,11 @@ Q4_DEVINL int ld_acquire(const int *p) {
 // __syncwarp() before each call orders the other lanes' writes first).
 Q4_DEVINL void red_release_add(int *p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+Q4_DEVINL int atom_acq_rel_cta_shared_add(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.cta.shared.add.s32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
 }
 Q4_DEVINL void tmap_acquire(const CUtensorMap *tm) {
     asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(tm) : "memory");
@@ -220,6 +225,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     uint64_t *empty = full + kRing;
     int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: a wait of this CTA gave up
     int *finq = flag + 4;  // [warp][2][4] pending sums of split row blocks: {entry, rb, parts, level}
+    int *pubq = finq + kConsumers * 8;  // [8] warps arrived at each of the last eight publications
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, G = a.G;
@@ -229,6 +235,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             mbar_init(empty + i, kConsumers);
         }
         flag[0] = 0;
+        for (int i = 0; i < 8; ++i) pubq[i] = 0;
         fence_barrier_init();
     }
     __syncthreads();
@@ -298,6 +305,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
         }
         float ys0 = 0.f, ys1 = 0.f;  // this lane's share of rows pr and pr + 8
         int slot = 0, round = 0;
+        int pub_j = 0;  // publications of this warp so far
         // split row blocks whose last part this CTA holds, by level parity: their sums (rows
         // of y) are written at the start of the level after next (see the file comment)
         int *fq = finq + warp * 8;
@@ -539,8 +547,19 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 // parts are published one tile late (their stores have landed by then, so the
                 // release does not stall), and at once at the end of the CTA's range
                 if (pend > 0 && (!block_end || i == n - 1)) {
+                    // every warp publishes the same parts in the same order: the warps count
+                    // their arrivals in shared memory and the last of the fifteen makes one
+                    // release increment for the CTA (its release carries what the other warps
+                    // wrote before their arrivals, which it acquired)
                     __syncwarp();
-                    if (lane == 0) red_release_add(a.parts_done + l, pend);
+                    if (lane == 0) {
+                        int *ctr = pubq + (pub_j & 7);
+                        if (atom_acq_rel_cta_shared_add(ctr, 1) == kConsumers - 1) {
+                            *ctr = 0;  // reused eight publications later; no warp is that far ahead
+                            red_release_add(a.parts_done + l, pend);
+                        }
+                    }
+                    ++pub_j;
                     pend = 0;
                 }
             }
@@ -715,7 +734,7 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
 
     // grid and shared memory
     const size_t fslot = bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>();  // B fragments + header of a tile
-    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4;
+    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4 + 8 * 4;
     if (fixed + fslot > (size_t)kSmemBudget) return Q4_ERR_UNSUPPORTED;
     int ucap = (int)((kSmemBudget - fixed) / fslot);
     if (ucap > kMaxUcap) ucap = kMaxUcap;
@@ -789,8 +808,8 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
             off += (size_t)pm * E.npad;
         }
         if (off > lo.part_floats) return Q4_ERR_WORKSPACE;  // cannot happen with grid <= kPlanGrid
-        if (pairs * kConsumers >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
-        lv.parts_target = (int)(pairs * kConsumers);
+        if (pairs >= ((int64_t)1 << 31)) return Q4_ERR_UNSUPPORTED;
+        lv.parts_target = (int)pairs;
         lv.fin_target = (int)split;
         for (int cc = 0; cc < grid; ++cc) {
             if (us[cc] == us[cc + 1]) continue;
