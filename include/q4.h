@@ -124,8 +124,9 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
  * digits, 2064 bytes per int4 stage and 1040 per int8 stage). One row of x needs none (0)
  * when each CTA's share of K, at most 4096, is built on chip. Groups of whole rows
  * (group a multiple of K) add N floats, rounded up to 256 bytes, at the start: their
- * scales spread to one per row. Same arguments as qgemm. Returns 0 for arguments qgemm
- * rejects. Depends only on the arguments, not on the device.
+ * scales spread to one per row. The any-group path needs none (0). Same arguments as
+ * qgemm. Returns 0 for arguments qgemm rejects. Depends only on the arguments, not on
+ * the device.
  */
 Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int64_t group,
                                 q4_xdtype xt);
@@ -136,8 +137,10 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * QuantizedMatmul of "Huit bits, puis quatre", section "Ranger des entiers
  * dans des f32": the same numbers as the product with the dequantized
  * weights, up to the order of the sums).
- *   x        [M][K], fp32 or bf16 per xt, row-major, 16-byte aligned
- *   payload  [N][K*bits/8] bytes from qpack of an [N][K] matrix, 16-byte aligned
+ *   x        [M][K], fp32 or bf16 per xt, row-major, 16-byte aligned (any
+ *            alignment of the element type on the any-group path below)
+ *   payload  q4_payload_bytes(N, K, bits) bytes from qpack of an [N][K] matrix,
+ *            16-byte aligned (any alignment on the any-group path)
  *   scales   [N*K/group] floats from the same qpack
  *   y        out, [M][N] fp32
  *   workspace  device scratch of at least q4_qgemm_workspace_bytes(...)
@@ -156,15 +159,19 @@ Q4_API size_t q4_qgemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits
  * pieces, or (one row of x, a 128-byte stage whose activations span at most 2^21)
  * as fixed-point digits within 2^-18 of each activation's own magnitude; the sums
  * are fp32. Activations below 2^-110 in magnitude may lose bits below 2^-133.
- * Requirements (else Q4_ERR_UNSUPPORTED): K % 32 == 0; group divides K with
- * group % 32 == 0 (per-channel scales are group = K), or group is a multiple
- * of K (groups of whole rows, down to one scale for the whole matrix, the
- * INT4_TENSOR format of the "量化推理：INT8/INT4 ..." page; N must then be a
- * multiple of group / K, else Q4_ERR_ARG). Groups of whole rows are spread to
- * one scale per row in the workspace by a first kernel, which the fused path
- * then reads (Q4_QGEMM_WEIGHTS_STATIC has no effect on such calls).
- * N, K <= 2^30 and M <= 1048560 (65535 chunks of 16 rows). M, N >= 0;
- * M == 0 or N == 0 enqueues nothing.
+ * Groups: every group qpack accepts (a divisor of N * K; int4 needs N * K even;
+ * else Q4_ERR_ARG). With K % 32 == 0 and a group that divides K in a multiple of 32
+ * (per-channel scales are group = K), or a multiple of K (groups of whole rows, down
+ * to one scale for the whole matrix, the INT4_TENSOR format of the "量化推理：
+ * INT8/INT4 ..." page), the paths above run; groups of whole rows are first spread
+ * to one scale per row in the workspace (Q4_QGEMM_WEIGHTS_STATIC has no effect on
+ * such calls). Any other group or K (g = 16, g = 48, g = 3K/2 crossing rows at a
+ * different offset in every row, odd K) runs on the any-group kernel: no workspace,
+ * exact fp32 w' as qdequant gives it, fp32 products and compensated fp32 sums
+ * (error <= 2^-20 * sum_k |w'x|); it is bound by its per-weight integer work, not
+ * by HBM.
+ * On the fused paths N, K <= 2^30 and M <= 1048560 (65535 chunks of 16 rows), else
+ * Q4_ERR_UNSUPPORTED. M, N >= 0; M == 0 or N == 0 enqueues nothing.
  * Errors: Q4_ERR_ARG (null pointers, bits, shapes), Q4_ERR_UNSUPPORTED,
  * Q4_ERR_WORKSPACE, Q4_ERR_CUDA.
  */

@@ -67,27 +67,46 @@ struct QgemmPlan {
     int64_t group;        // group the kernels see: the caller's, or K for groups of whole rows
     int64_t rps;          // rows per scale when the group spans whole rows, else 1
     bool prefill;         // bf16 x, M >= 64: the tensor-core GEMM
+    bool any;             // a group neither fast path takes: the any-group kernel (no workspace)
     size_t scale_bytes;   // expanded per-row scales at the start of the workspace (rps > 1)
     size_t total_bytes;   // workspace the call needs
 };
 
-// Returns Q4_OK and fills the plan, or the reason the call cannot run. Groups either divide
-// K, or are whole multiples of K (c rows share a scale; their scales are first expanded to
-// one per row in the workspace).
+// Returns Q4_OK and fills the plan, or the reason the call cannot run. Groups that divide
+// K (in multiples of 32) run on the fused GEMV or the tensor-core GEMM; groups of whole
+// rows too, once their scales are expanded to one per row in the workspace; every other
+// divisor of N * K (and any K) runs on the any-group kernel.
 q4_status plan_qgemm(int64_t M, int64_t N, int64_t K, int bits, int64_t group, q4_xdtype xt, QgemmPlan *p) {
     if (bits != 4 && bits != 8) return Q4_ERR_ARG;
     if (M < 0 || N < 0 || K < 1 || group < 1) return Q4_ERR_ARG;
     if (xt != Q4_X_F32 && xt != Q4_X_BF16) return Q4_ERR_ARG;
+    if (N > 0 && (N > ((int64_t)1 << 40) / K || (N * K) % group != 0)) return Q4_ERR_ARG;  // no such packed tensor
+    if (bits == 4 && (N * K) % 2 != 0) return Q4_ERR_ARG;                               // (qpack's rule)
     p->group = group;
     p->rps = 1;
+    p->any = false;
+    p->prefill = false;
     if (K % group != 0) {
-        if (group % K != 0) return Q4_ERR_UNSUPPORTED;
-        p->rps = group / K;
-        if (N % p->rps != 0) return Q4_ERR_ARG;  // no [N][K] matrix has such groups
-        p->group = K;
+        if (group % K == 0) {
+            p->rps = group / K;
+            p->group = K;
+        } else {
+            p->any = true;
+        }
     }
-    if (!q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, p->group, xt == Q4_X_BF16, kPlanSMs, &p->gemv))
+    // the fused paths take K and groups in multiples of 32 (groups of whole rows as K)
+    if (!p->any && (K % 32 != 0 || p->group % 32 != 0)) {
+        p->any = true;
+        p->group = group;
+        p->rps = 1;
+    }
+    if (!p->any && !q4::gemv_plan(M > 0 ? M : 1, N > 0 ? N : 1, K, bits, p->group, xt == Q4_X_BF16, kPlanSMs,
+                                  &p->gemv))
         return Q4_ERR_UNSUPPORTED;
+    if (p->any) {
+        p->scale_bytes = p->total_bytes = 0;
+        return Q4_OK;
+    }
     p->prefill = q4::prefill_supported(M, N, K, bits, p->group, xt == Q4_X_BF16);
     p->scale_bytes = p->rps > 1 ? align256((size_t)N * 4) : 0;
     p->total_bytes = p->scale_bytes + (p->prefill ? 0 : p->gemv.bytes);
@@ -193,6 +212,11 @@ q4_status qgemm_ex(const void *x, q4_xdtype xt, int64_t M, const uint8_t *payloa
     if (st != Q4_OK) return st;
     if (M == 0 || N == 0) return Q4_OK;
     if (!x || !payload || !scales || !y) return Q4_ERR_ARG;
+    if (p.any) {
+        const cudaError_t ae = q4::launch_any_group(x, xt == Q4_X_BF16, M, payload, scales, N, K, bits, group, y,
+                                                    device_sms(), as_stream(stream));
+        return cuda_status(ae, "any-group launch");
+    }
     if ((uintptr_t)payload % 16 || (uintptr_t)x % 16) return Q4_ERR_UNSUPPORTED;
     if ((!p.prefill || p.total_bytes > 0) && (uintptr_t)workspace % 256) return Q4_ERR_WORKSPACE;
     if (p.total_bytes > 0 && (!workspace || workspace_bytes < p.total_bytes)) return Q4_ERR_WORKSPACE;

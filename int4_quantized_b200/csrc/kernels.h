@@ -71,4 +71,10 @@ cudaError_t launch_prefill(const void *x, int64_t M, const uint8_t *payload, con
                            int64_t K, int bits, int64_t group, float *y, uint32_t *status, int sms,
                            cudaStream_t st);
 
+// ---- any group (anygroup.cu) ------------------------------------------------------------
+// Groups the two paths above do not take: any divisor of N * K (crossing rows at varying
+// offsets, or narrower than 32), any K; exact fp32 w', fp64 sums.
+cudaError_t launch_any_group(const void *x, bool x_bf16, int64_t M, const uint8_t *payload, const float *scales,
+                             int64_t N, int64_t K, int bits, int64_t group, float *y, int sms, cudaStream_t st);
+
 }  // namespace q4

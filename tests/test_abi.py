@@ -77,11 +77,10 @@ def test_qpack_validation(q4, rows, cols, bits, group, ptr_ok, expect):
     (1, 64, 128, 3, 128, 0, 1),     # bits
     (1, 64, 128, 4, 0, 0, 1),       # group
     (1, 64, 128, 4, 128, 7, 1),     # x dtype
-    (1, 64, 96, 4, 64, 0, 2),       # group does not divide K
-    (1, 64, 48, 4, 48, 0, 2),       # K % 32
-    (1, 64, 128, 4, 16, 0, 2),      # int4 group % 32
-    (1, 64, 128, 8, 8, 0, 2),       # int8 group % 32
-    (1, 64, 128, 8, 16, 0, 2),      # int8 group % 32
+    (1, 64, 96, 4, 5, 0, 1),        # group does not divide N * K
+    (1, 3, 3, 4, 3, 0, 1),          # an odd number of int4 weights
+    (1, 64, 128, 4, 128 * 65, 0, 1),  # whole-row groups that do not divide N
+    (65535 * 16 + 1, 64, 128, 4, 128, 0, 2),  # more rows of x than the fused GEMV takes
     (-1, 64, 128, 4, 128, 0, 1),    # negative M
 ])
 def test_qgemm_validation(q4, M, N, K, bits, group, xt, expect):
@@ -114,7 +113,8 @@ def test_qgemm_ex_flags_and_limits(q4):
     for flags in (2, 4, 0x80000000):
         assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need, flags, None, None) == 1
     # with the static-weights flag the argument rules are those of qgemm
-    assert lib.qgemm_ex(FAKE, 0, 1, FAKE, FAKE, 64, 128, 4, 16, FAKE, None, 0, 1, None, None) == 2
+    assert lib.qgemm_ex(FAKE, 0, 65535 * 16 + 1, FAKE, FAKE, 64, 128, 4, 128, FAKE, None, 0, 1, None, None) == 2
+    assert lib.qgemm_ex(FAKE, 0, 1, FAKE, FAKE, 64, 128, 4, 5, FAKE, None, 0, 1, None, None) == 1
     assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, 1, None, None) == 5
     assert lib.qgemm_ex(None, 0, 0, None, None, 4096, 4096, 4, 128, None, None, 0, 1, None, None) == 0
     # rows of x: at most 65535 chunks of 16
@@ -133,9 +133,9 @@ def test_groups_of_whole_rows(q4):
         assert q4.qgemm_workspace_bytes(300, N, K, 4, g, torch.bfloat16) == 256  # the GEMM needs only those
         assert q4.qgemm_workspace_bytes(8, N, K, 8, g) == 256 + q4.qgemm_workspace_bytes(8, N, K, 8, K)
     assert q4.qgemm_workspace_bytes(1, 1000, K, 4, K * 1000) == 4096
-    # groups that neither divide K nor are whole rows; N not a multiple of the rows per group
+    # groups that do not divide N * K: no packed tensor has them
     ok = ctypes.c_void_p(0x100000)
-    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, 3 * K // 2, FAKE, ok, 1 << 20, None, None) == 2
+    assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, 3 * K // 2, FAKE, ok, 1 << 20, None, None) == 1
     assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, 63, K, 4, 2 * K, FAKE, ok, 1 << 20, None, None) == 1
     # the spread scales must fit in the workspace
     assert lib.qgemm(FAKE, 0, 1, FAKE, FAKE, N, K, 4, N * K, FAKE, ok, 255, None, None) == 5
@@ -147,3 +147,21 @@ def test_workspace_is_a_pure_function_of_the_problem(q4):
         a = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)
         b = q4.qgemm_workspace_bytes(M, 11008, 4096, 4, 128)
         assert a == b and a % 256 == 0
+
+
+def test_any_group_is_planned(q4):
+    # every group qpack accepts plans (M = 0 returns Q4_OK only after the plan accepted the
+    # shape): narrow groups dividing K, groups crossing rows at varying offsets, odd K; the
+    # any-group path needs no workspace
+    import torch
+
+    lib = q4.lib()
+    for N, K, bits, g in [(64, 256, 4, 16), (96, 256, 8, 48), (66, 256, 4, 384), (30, 77, 4, 10),
+                          (7, 3, 8, 7), (33, 100, 4, 50), (64, 96, 4, 1), (12, 100, 8, 100)]:
+        assert lib.qgemm(None, 0, 0, None, None, N, K, bits, g, None, None, 0, None, None) == 0, (N, K, g)
+        assert q4.qgemm_workspace_bytes(1, N, K, bits, g) == 0
+        assert q4.qgemm_workspace_bytes(100, N, K, bits, g, torch.bfloat16) == 0
+    # not a divisor of N * K, or an odd number of int4 weights: no such payload
+    assert lib.qgemm(None, 0, 0, None, None, 30, 77, 4, 4, None, None, 0, None, None) == 1
+    assert lib.qgemm(None, 0, 0, None, None, 7, 3, 4, 7, None, None, 0, None, None) == 1
+    assert lib.qgemm(None, 0, 0, None, None, 7, 3, 8, 7, None, None, 0, None, None) == 0

@@ -247,3 +247,38 @@ def test_groups_of_whole_rows(q4, bits, rows_per_group, M, bf16):
     check(y.cpu().numpy(), yref, bound, f"int{bits} g{g} M{M}")
     assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
     assert torch.equal(y.view(torch.int32), y3.view(torch.int32))
+
+
+ANY_GROUP = [
+    # M, N, K, bits, group, bf16 x -- groups the fused paths do not take
+    (1, 64, 256, 4, 16, False),       # narrower than a 32-wide segment
+    (3, 96, 256, 8, 48, False),       # 48 does not divide K: groups cross rows at varying offsets
+    (5, 66, 256, 4, 384, False),      # 3K/2: every other row starts mid-group
+    (2, 30, 77, 4, 10, False),        # odd K: int4 rows start in the middle of a byte
+    (1, 7, 3, 8, 7, False),           # groups longer than a row, tiny
+    (17, 33, 100, 4, 50, True),       # K % 32 != 0, bf16 x
+    (70, 64, 96, 4, 1, True),         # one scale per weight, many rows of x
+    (9, 12, 100, 8, 100, False),      # per-row scales with K % 32 != 0
+    (1, 257, 1000, 4, 40, False),     # groups of 40 crossing rows, ragged sizes
+    (8, 2048, 2048, 4, 16, False),    # a larger one (scales of 16 weights)
+]
+
+
+@pytest.mark.parametrize("idx", range(len(ANY_GROUP)))
+def test_any_group(q4, idx):
+    # every group that qpack accepts, through the any-group kernel, against the oracle's
+    # dequantization of the flattened tensor (groups cut across rows as pack() cuts them)
+    M, N, K, bits, g, bf16 = ANY_GROUP[idx]
+    rng = np.random.default_rng(700 + idx)
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    payload, scales, _ = oracle.pack(w, bits, g)
+    xin = x
+    if bf16:
+        import torch
+
+        xin = torch.from_numpy(x).to(torch.bfloat16).float().numpy()  # the values the GPU reads
+    y = run_gpu(q4, x, payload, scales, N, K, bits, g, bf16=bf16)
+    yref, bound = oracle.qgemm(xin, payload, scales, N, K, bits, g)
+    check(y, yref, bound, f"any group M={M} N={N} K={K} int{bits} g={g}")
+    assert q4.qgemm_workspace_bytes(M, N, K, bits, g) == 0
