@@ -14,15 +14,17 @@
 // epilogue warps add scale * partial into fp32 registers ("promotion"), so the result is
 // the fp32 product of exact codes and activations, rounded only by fp32 sums.
 //
-// Warp roles (384 threads, one CTA per SM, persistent over output tiles):
+// Warp roles (512 threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: x tile (256 x 64 bf16) and payload tile (128 rows) per k-step
 //               into a 4-deep ring (full/empty mbarriers);
 //   warp 1      allocates tensor memory; one lane issues the MMAs (4 per k-step) and the
 //               tcgen05.commit arrivals that free ring slots and publish finished groups;
-//   warps 2-3   dequantize the payload tile (two rows per thread) into a 3-deep ring of A
-//               tiles, made visible to the tensor core with fence.proxy.async;
-//   warps 4-11  epilogue: warp w reads tensor-memory lanes 32*(w%4).. and 128 of the 256
+//   warps 2-5   dequantize the payload tile (one row per thread) into a 3-deep ring of A
+//               tiles, made visible to the tensor core with fence.proxy.async (warps 6-7
+//               have no role: they fill the second warpgroup);
+//   warps 8-15  epilogue: warp w reads tensor-memory lanes 32*(w%4).. and 128 of the 256
 //               columns, keeps them as fp32 accumulators, stores y at the end of a tile.
+// Registers move from the first two warpgroups to the epilogue ones (setmaxnreg).
 // With one scale per output channel (one group per tile) the scale is applied once at the
 // end, the epilogue needs no accumulators and 4 warps (10-13), and warps 2-9 dequantize
 // (consecutive threads take consecutive 16-byte chunks of the payload tile).
@@ -42,7 +44,13 @@ constexpr int kBN = 256;          // activation rows per tile (MMA N)
 constexpr int kBK = 64;           // k per step: one 128-byte swizzle row of bf16
 constexpr int kStages = 4;        // x + payload ring
 constexpr int kAStages = 3;       // dequantized A ring
-constexpr int kThreads = 384;     // grouped scales: TMA, MMA, 2 dequantizing, 8 epilogue warps
+constexpr int kThreads = 512;     // grouped scales: TMA, MMA, 4 dequantizing, 2 idle, 8 epilogue warps
+// Grouped scales: the kernel launches at kRegsLaunch registers a thread; the first two
+// warpgroups (TMA, MMA, dequantizing) give theirs down to kRegsLow and the two epilogue
+// warpgroups (128 fp32 accumulators a thread) take kRegsHigh: 256 * 64 + 256 * 192 is
+// exactly the 512 * 128 the block holds, so every increase is served.
+constexpr int kRegsLaunch = 128, kRegsLow = 64, kRegsHigh = 192;
+static_assert(4 * 32 * 2 * kRegsLow + 4 * 32 * 2 * kRegsHigh == kThreads * kRegsLaunch, "register split");
 constexpr int kThreadsPC = 448;   // one scale per output channel: TMA, MMA, 8 dequantizing, 4 epilogue
 constexpr int kXBytes = kBN * kBK * 2;        // 32 KB
 constexpr int kABytes = kBM * kBK * 2;        // 16 KB
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(PC ? kThreadsPC : kThreads, 1)
 prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmp) {
     constexpr int PB = kBM * kBK * BITS / 8;  // payload bytes per k-step (4 or 8 KB)
     constexpr int PROW = kBK * BITS / 8;      // payload bytes per row per k-step (32 or 64)
-    constexpr int NDQW = PC ? 8 : 2;          // dequantizing warps (warps 2 .. 1 + NDQW)
+    constexpr int NDQW = PC ? 8 : 4;          // dequantizing warps (warps 2 .. 1 + NDQW)
     constexpr int NCH = PROW / 16;            // 16-byte payload chunks per row and k-step
     constexpr int UPT = kBM * NCH / (32 * NDQW);  // payload chunks per dequantizing thread
     constexpr int NEPW = PC ? 4 : 8;          // epilogue warps (the rest)
@@ -232,7 +240,7 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
     bool timed_out = false;
     const int ntile_cta = a.items > (int)blockIdx.x ? (a.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-    if (warp == 0) {
+    auto tma_role = [&]() {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int it = 0;
@@ -251,7 +259,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 if (timed_out) break;
             }
         }
-    } else if (warp == 1) {
+    };
+    auto mma_role = [&]() {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             int it = 0, ait = 0, grp = 0;
@@ -283,7 +292,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
             }
             umma_commit(done);
         }
-    } else if (warp < 2 + NDQW) {
+    };
+    auto dequant_role = [&]() {
         // ---------------- dequantize: payload -> bf16 codes (A) ----------------
         const int dt = threadIdx.x - 64;  // payload chunks dt + 32 * NDQW * i, i < UPT
         int it = 0, ait = 0;
@@ -321,21 +331,27 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                         }
                     }
                 } else {
-                    // two whole rows per thread (rows dt and dt + 64)
+                    // whole rows: row dt (and dt + 32 * NDQW, ... while rows remain)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int r = dt + 64 * h;
+                    for (int h = 0; h < kBM / (32 * NDQW); ++h) {
+                        const int r = dt + 32 * NDQW * h;
                         const uint4 *src = reinterpret_cast<const uint4 *>(pst + r * PROW);
                         uint8_t *dst = ast + r * 128;
+                        // rows sit 32 (int4) or 64 (int8) bytes apart, so the lanes of one
+                        // shared-memory phase would read the same banks; each lane starts at a
+                        // chunk that depends on its row, which spreads them over all banks
                         if constexpr (BITS == 4) {
-                            const uint4 p0 = src[0], p1 = src[1];  // 64 codes
+                            const int j0 = (r >> 2) & 1;  // rows r and r + 4 take different halves first
+                            const uint4 pa = src[j0], pb = src[j0 ^ 1];
+                            const uint4 p0 = j0 ? pb : pa, p1 = j0 ? pa : pb;  // 64 codes
                             const uint32_t wds[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
                             for (int c = 0; c < 8; ++c)
                                 *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = codes_int4(wds[c]);
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
+                            for (int c0 = 0; c0 < 8; ++c0) {
+                                const int c = (c0 + r) & 7;
                                 const uint2 wv = reinterpret_cast<const uint2 *>(src)[c];  // 8 codes
                                 const uint2 lo = codes_int8(wv.x), hi = codes_int8(wv.y);
                                 *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) =
@@ -352,7 +368,8 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 }
             }
         }
-    } else if constexpr (PC) {
+    };
+    auto epilogue_pc = [&]() {
         // ---------------- epilogue, one group per tile: y = scale * D ----------------
         const int q = warp & 3;
         const int rl = 32 * q + lane;
@@ -384,9 +401,10 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
             __syncwarp();
             if (lane == 0) mbar_arrive(dempty + d);
         }
-    } else {
+    };
+    auto epilogue_grouped = [&]() {
         // ---------------- epilogue: promotion and stores ----------------
-        const int q = warp & 3, half = (warp - 4) >> 2;
+        const int q = warp & 3, half = (warp - 8) >> 2;
         const int rl = 32 * q + lane;                       // weight row inside the tile
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half);
         int grp = 0;
@@ -436,7 +454,31 @@ prefill_gemm(const PrefillArgs a, const __grid_constant__ CUtensorMap tmx, const
                 }
             }
         }
+    };
+    if constexpr (PC) {
+        if (warp == 0)
+            tma_role();
+        else if (warp == 1)
+            mma_role();
+        else if (warp < 2 + NDQW)
+            dequant_role();
+        else
+            epilogue_pc();
+    } else if (warp < 8) {
+        // the first two warpgroups give registers up, at one program point for all 8 warps
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+        if (warp == 0)
+            tma_role();
+        else if (warp == 1)
+            mma_role();
+        else if (warp < 2 + NDQW)
+            dequant_role();
+        // warps 6 and 7: no role
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+        epilogue_grouped();
     }
+
 
     // wait for the last MMAs before releasing tensor memory
     if (warp == 1 && lane == 0 && !timed_out) timed_out = !mbar_wait(done, 0);
@@ -511,6 +553,19 @@ cudaError_t launch_prefill(const void *x, int64_t M, const uint8_t *payload, con
                           : (pc ? prefill_gemm<8, true> : prefill_gemm<8, false>);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
+    if (!pc) {
+        // the register split above assumes the block launches at exactly kRegsLaunch a
+        // thread; any other allocation could leave an increase waiting: refuse to launch
+        static int regs[2] = {0, 0};
+        int &rg = regs[bits == 4 ? 0 : 1];
+        if (!rg) {
+            cudaFuncAttributes fa;
+            const cudaError_t ae = cudaFuncGetAttributes(&fa, kern);
+            if (ae != cudaSuccess) return ae;
+            rg = fa.numRegs;
+        }
+        if (rg != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    }
     kern<<<grid, pc ? kThreadsPC : kThreads, smem, st>>>(a, tmx, tmp);
     return cudaGetLastError();
 }
