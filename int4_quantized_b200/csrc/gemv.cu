@@ -62,6 +62,7 @@ constexpr int kPayloadBytes = kTileBytes * kRowsPerCta;  // 16 KB of codes per s
 constexpr int kMaxStages = 6;
 constexpr int kGroupsPerBlock = 8;                 // scale groups per k-block (target)
 constexpr int kBlockK = 1024;                      // at most k per k-block
+constexpr int kPrepSplit = 8;                      // gemv_prep CTAs per k-block (several rows of x)
 constexpr int kSG = 12;                            // scale slots per row per k-block (<= 9 used,
                                                    // + up to 3 to keep 16-byte copies aligned)
 constexpr int kInkMaxK = 4096;                     // k of one CTA's range whose pieces are built on
@@ -129,16 +130,19 @@ __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
             build_slot1<BITS, L, XBF16, false>(a.frag + (size_t)s * a.fslot_bytes, a.x, s * STAGEK, a.K, a.P, lane);
         return;
     }
-    const int eb = blockIdx.x, mc = blockIdx.y;
+    // several rows: kPrepSplit CTAs share a k-block (an item, 8 k of one row, per thread
+    // or two), so the loads of x are in flight together
+    const int eb = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit, mc = blockIdx.y;
     const int mcnt = min(16, a.M - mc * 16);
     const int ncols = stored_cols(a.NB, a.lw);
     const int vrows = (ncols + a.P - 1) / a.P;
     const int k0 = eb * a.ebs * STAGEK;
     const int k1 = min(a.K, k0 + a.ebs * STAGEK);
     const int nu = (k1 - k0) / 8;  // 8-k units in the block (at most 128)
+    const int u_lo = part * nu / kPrepSplit, nun = (part + 1) * nu / kPrepSplit - u_lo;
     uint2 *fbase = reinterpret_cast<uint2 *>(a.frag) + (size_t)mc * a.stages_total * (a.fslot_bytes / 8);
-    for (int it = threadIdx.x; it < nu * vrows; it += blockDim.x) {
-        const int vm = it / nu, u = it - vm * nu;
+    for (int it = threadIdx.x; it < nun * vrows; it += blockDim.x) {
+        const int vm = it / nun, u = u_lo + (it - vm * nun);
         const int k = k0 + 8 * u;
         float v[8];
         if (vm < mcnt) {
@@ -572,7 +576,7 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
     if (NB > 4) early = false;
     if constexpr (!INK) {
         cudaLaunchConfig_t pc = {};
-        pc.gridDim = dim3(pl.n_eb, pl.nmc);
+        pc.gridDim = dim3(HYB ? pl.n_eb : pl.n_eb * kPrepSplit, pl.nmc);
         pc.blockDim = dim3(256);
         pc.stream = st;
         pc.attrs = &pdl;
