@@ -62,8 +62,13 @@ constexpr int kConsumerThreads = 32 * kConsumers;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSRows = 16 * kConsumers;            // 240 weight rows per tile
 constexpr int kSTile = kTileBytes * kSRows;        // 30 KB of codes per tile
-constexpr int kRing = 4;                           // tiles in flight per CTA
-constexpr int kSmemBudget = 163840;
+// Tiles in flight per CTA, and the shared memory the CTA takes: with several scale groups
+// per tile the consumers' scale lines need about 70 KB of L1 (4 tiles, 160 KB of shared
+// memory); with one scale per stage or per row they need little, and a fifth tile in
+// flight pays (172 KB).
+__host__ __device__ constexpr int ring_of(int gps) { return gps > 0 ? 4 : 5; }
+constexpr int smem_budget_of(int gps) { return gps > 0 ? 163840 : 174080; }
+constexpr int ucap_max_of(int gps) { return gps > 0 ? 64 : 10; }
 constexpr int kCtasPerSm = 1;
 
 struct alignas(64) StackEntry {
@@ -177,7 +182,6 @@ Q4_DEVINL bool wait_counter(const int *p, int target, uint64_t limit_ns) {
     }
 }
 
-constexpr int kMaxUcap = 64;  // tiles whose slots are built at once, at most
 #ifndef Q4_STACK_MAX_READ_PARTS
 #define Q4_STACK_MAX_READ_PARTS 1000
 #endif
@@ -219,6 +223,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     constexpr int FSLOT = slot1_bytes<BITS>();  // B fragments of one tile + format header
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    constexpr int kRing = ring_of(GPS);
     uint8_t *ring = smem;                                                  // kRing x 30 KB
     uint8_t *bbuf = ring + kRing * kSTile;                             // ucap x FSLOT
     uint64_t *full = reinterpret_cast<uint64_t *>(bbuf + (size_t)a.ucap * FSLOT);
@@ -295,7 +300,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     } else {
         // ---------------- consumers ----------------
         const int g = lane >> 2, t = lane & 3;
-        const int ct = threadIdx.x;
+
         const int pr = 16 * warp + row_perm<L>(g);
         uint32_t aoff[SPS];
 #pragma unroll
@@ -734,10 +739,12 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
 
     // grid and shared memory
     const size_t fslot = bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>();  // B fragments + header of a tile
+    const int kRing = ring_of(lo.gps);
+    const size_t budget = (size_t)smem_budget_of(lo.gps);
     const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4 + 8 * 4;
-    if (fixed + fslot > (size_t)kSmemBudget) return Q4_ERR_UNSUPPORTED;
-    int ucap = (int)((kSmemBudget - fixed) / fslot);
-    if (ucap > kMaxUcap) ucap = kMaxUcap;
+    if (fixed + fslot > budget) return Q4_ERR_UNSUPPORTED;
+    int ucap = (int)((budget - fixed) / fslot);
+    if (ucap > ucap_max_of(lo.gps)) ucap = ucap_max_of(lo.gps);
     const size_t smem = fixed + (size_t)ucap * fslot;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_error(e, "stack kernel attribute");
