@@ -539,6 +539,30 @@ def mlp70b_section(args, dev, peaks):
         gbs = nb / (us * 1e-6) / 1e9
         out["int4_g64_static" if static else "int4_g64"] = {"us_per_matrix": round(us, 2), "GB/s": round(gbs, 1),
                                                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    # the same three matrices as one MLP step in the persistent decode-stack kernel: gate and
+    # up read x (level 0), down reads gate's output (level 1); one launch per step
+    (mg, pg, sg, xg, yg), (mu, pu, su, xu, yu), (md, pd, sd, _, yd) = mats
+    st = q4.DecodeStack([q4.StackGemv(pg, sg, xg.reshape(-1), yg.reshape(-1), mg.N, mg.K, group, 0),
+                         q4.StackGemv(pu, su, xg.reshape(-1), yu.reshape(-1), mu.N, mu.K, group, 0),
+                         q4.StackGemv(pd, sd, yg.reshape(-1), yd.reshape(-1), md.N, md.K, group, 1)], bits)
+    stream = torch.cuda.Stream(device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            st.run(status)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(20):
+            st.run(status)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError("a bounded wait in the decode-stack kernel gave up")
+    us = e0.elapsed_time(e1) * 1e3 / 20
+    gbs = 3 * nb / (us * 1e-6) / 1e9
+    out["int4_g64_persistent_mlp"] = {"us_per_step": round(us, 2), "us_per_matrix": round(us / 3, 2),
+                                      "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                      "kernel": "decode stack: gate|up (level 0), down reading gate's output (level 1)"}
     return out
 
 
