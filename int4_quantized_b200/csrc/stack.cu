@@ -27,10 +27,11 @@
 //     previous-level GEMV's y, the next level reads x as the sum of that slice's parts
 //     (in part order; absent parts are zeros). The y of a split row block is written by
 //     the CTA holding its last part, as the same sum, so y and what the next level read
-//     are the same numbers; it does so at the start of the level after next, while it
-//     waits for the level before to end (at the next start if the next level reads that
-//     y directly). A level waits for the sums of three levels back (the parts buffers
-//     rotate over three levels) and of every earlier level whose y it reads directly.
+//     are the same numbers; it does so at the start of the level after next, on the warps
+//     that have no slot to build while the others build (at the next start, before the
+//     build, if the next level reads that y directly). A level waits for the sums of three
+//     levels back (the parts buffers rotate over three levels) and of every earlier level
+//     whose y it reads directly.
 //   * Counters return to zero at the end of every launch (the last CTA to finish resets
 //     them), so the workspace can be replayed, e.g. from a CUDA graph.
 //
@@ -54,9 +55,9 @@ namespace {
 using namespace gm;
 
 // One CTA per SM: fifteen consumer warps (16 weight rows each) on 240-row tiles and one
-// producer warp. Registers: 512 threads x 128 fill the SM's 64K; shared memory stays near
-// 160 KB so that about 70 KB of the SM's 228 KB remain L1, which holds the lines of scales
-// the consumers read (a 128-byte line serves a row over many consecutive stages).
+// producer warp. Registers: 512 threads x 128 fill the SM's 64K. The consumers read scales
+// through L1 (a 128-byte line serves a row over many consecutive stages), so shared memory
+// leaves room for it (below).
 constexpr int kConsumers = 15;
 constexpr int kConsumerThreads = 32 * kConsumers;
 constexpr int kThreads = kConsumerThreads + 32;

@@ -226,6 +226,68 @@ def test_llama7b_stack_sampled(q4):
         assert np.all(err <= RTOL * bound + ATOL), f"GEMV {idx}: worst ratio {(err / (RTOL * bound + ATOL)).max():.3g}"
 
 
+def test_llama7b_int8_per_channel_sampled(q4):
+    # the full step at int8 with one scale per output channel (6.5 GB): the kernel variant
+    # with five tiles in flight, whose CTAs build the slots of q|k|v and gate|up in several
+    # chunks (more tiles per CTA than fit at once)
+    import torch
+
+    from int4_quantized_b200 import decode_stack as ds
+
+    stack = ds.build_stack(8, None, 32, torch.device("cuda"))
+    dstack, acts = ds.make_decode_stack(stack, 8)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        dstack.run(status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rng = np.random.default_rng(1)
+    for idx in (0, 2, 4, 6, 7 * 17 + 4, 7 * 31 + 6):
+        g = dstack.gemvs[idx]
+        N, K = g.N, g.K
+        p = g.payload.cpu().numpy()
+        s = g.scales.cpu().numpy()
+        rows = sorted(set(rng.choice(N, 48, replace=False).tolist()) | {0, N - 1})
+        x = g.x.float().cpu().numpy().reshape(1, K)
+        yref, bound = oracle.qgemm(x, p, s, N, K, 8, K, rows=rows)
+        y = g.y.cpu().numpy()[rows].astype(np.float64).reshape(1, -1)
+        err = np.abs(y - yref)
+        assert np.all(err <= RTOL * bound + ATOL), f"GEMV {idx}: worst ratio {(err / (RTOL * bound + ATOL)).max():.3g}"
+
+
+def test_slots_built_in_chunks(q4):
+    # a level of 28672 x 8192 int4 g128 gives each CTA about 26 tiles, more than the slots
+    # that fit in shared memory at once: the CTA builds them chunk by chunk; the next level
+    # reads the first 8192 outputs through their parts
+    import torch
+
+    rng = np.random.default_rng(41)
+    N1, K1, N2 = 28672, 8192, 1024
+    w1 = rng.normal(0, 1 / np.sqrt(K1), (N1, K1)).astype(np.float32)
+    w2 = rng.normal(0, 1 / np.sqrt(K1), (N2, K1)).astype(np.float32)
+    p1, s1, _ = oracle.pack(w1, 4, 128)
+    p2, s2, _ = oracle.pack(w2, 4, 128)
+    del w1, w2
+    x = torch.from_numpy(rng.normal(0, 1, K1).astype(np.float32)).cuda()
+    y1 = torch.empty(N1, device="cuda")
+    y2 = torch.empty(N2, device="cuda")
+    gemvs = [q4.StackGemv(torch.from_numpy(p1).cuda(), torch.from_numpy(s1).cuda(), x, y1, N1, K1, 128, 0),
+             q4.StackGemv(torch.from_numpy(p2).cuda(), torch.from_numpy(s2).cuda(), y1[:K1], y2, N2, K1, 128, 1)]
+    st = q4.DecodeStack(gemvs, 4)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st.run(status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows1 = sorted(set(rng.choice(N1, 96, replace=False).tolist()) | {0, N1 - 1})
+    for g, pk, sk, N, rows in ((gemvs[0], p1, s1, N1, rows1), (gemvs[1], p2, s2, N2, None)):
+        xh = g.x.float().cpu().numpy().reshape(1, K1)
+        yref, bound = oracle.qgemm(xh, pk, sk, N, K1, 4, 128, rows=rows)
+        y = g.y.cpu().numpy()
+        y = (y if rows is None else y[rows]).astype(np.float64).reshape(1, -1)
+        err = np.abs(y - yref)
+        assert np.all(err <= RTOL * bound + ATOL), f"worst ratio {(err / (RTOL * bound + ATOL)).max():.3g}"
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 def test_stages_of_every_activation_range(q4, bits):
     # per 128-byte stage the kernel takes exact integer digits when the stage's activations
