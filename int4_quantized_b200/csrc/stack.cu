@@ -98,8 +98,9 @@ struct StackLevel {
     int parts_target;      // parts that complete the level (one arrival per part)
     int fin_target;        // arrivals that complete its sums of split row blocks: one per block
     int fin_lo, fin_hi;    // levels whose sums must be in y before this level starts (none: lo > hi)
-    int needs_final;       // it reads a y of the previous level other than as a slice of parts
-    int fin_early;         // the next level reads its y other than as parts: sums at the next start
+    int needs_final;       // the previous level's sums go to y at this level's start: it reads
+                           // that y other than as a slice of parts, or the next level reads
+                           // the y of the level before it
 };
 
 struct StackArgs {
@@ -328,9 +329,17 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             for (int rr = (warp - w0) * 32 + lane; rr < kSRows; rr += nw * 32) {
                 const int row = f[1] * kSRows + rr;
                 if (row < fe->N) {
+                    // four loads in flight at a time, added in part order
                     const float *pp = fe->parts + row;
-                    float v = __ldcg(pp);
-                    for (int q = 1; q < np; ++q) v += __ldcg(pp + q * st);
+                    float v = 0.f;
+                    for (int q0 = 0; q0 < np; q0 += 4) {
+                        float pv[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) pv[j] = q0 + j < np ? __ldcg(pp + (q0 + j) * st) : 0.f;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (q0 + j < np) v = q0 + j == 0 ? pv[0] : v + pv[j];
+                    }
                     if (np < fe->pmax) v += 0.f;  // as the sum over all pmax parts, zeros included
                     fe->y[row] = v;
                 }
@@ -853,7 +862,6 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
                     P.is_src = 1;
                 } else {
                     lev[l].needs_final = 1;
-                    lev[l - 1].fin_early = 1;
                 }
             } else {
                 StackLevel &lv = lev[l];
@@ -863,6 +871,9 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
                     lv.fin_lo = std::min(lv.fin_lo, P.level);
                     lv.fin_hi = std::max(lv.fin_hi, P.level);
                 }
+                // the sums of level l - 2 are otherwise written at the start of level l,
+                // after its wait for them: level l - 1 writes them at its start instead
+                if (P.level == l - 2) lev[l - 1].needs_final = 1;
             }
         }
     }

@@ -372,3 +372,37 @@ def test_x_read_as_slices_of_earlier_outputs(q4):
     assert int(status.item()) == 0
     assert float(Y[1000]) == 0.0  # nobody writes between the two outputs
     check_all(gemvs, host, 4, "slices")
+
+
+def test_y_of_two_levels_back_read_directly(q4):
+    # level 2 reads A's y (level 0) directly while level 1 reads A only through its parts:
+    # A's sums must be in y before level 2 waits for them (level 1 writes them at its start)
+    import torch
+
+    rng = np.random.default_rng(37)
+    h = torch.from_numpy(rng.normal(0, 1, 1024).astype(np.float32)).cuda()
+    yA = torch.empty(1000, dtype=torch.float32, device="cuda")
+    yC = torch.empty(300, dtype=torch.float32, device="cuda")
+    spec = [  # name, N, K, level, x
+        ("A", 1000, 1024, 0, h),
+        ("C", 300, 512, 1, yA[0:512]),   # through A's parts
+        ("F", 200, 512, 2, yA[256:768]),  # A's y itself
+        ("G", 96, 256, 2, yC[0:256]),    # through C's parts
+    ]
+    outs = {"A": yA, "C": yC}
+    gemvs, host = [], []
+    for name, N, K, lvl, x in spec:
+        w = rng.normal(0, 1.0 / np.sqrt(K), (N, K)).astype(np.float32)
+        p, s, _ = oracle.pack(w, 4, 128)
+        y = outs.get(name)
+        if y is None:
+            y = torch.empty(N, dtype=torch.float32, device="cuda")
+        gemvs.append(q4.StackGemv(torch.from_numpy(p).cuda(), torch.from_numpy(s).cuda(), x, y, N, K, 128, lvl))
+        host.append((name, lvl, N, K, 128, p, s))
+    st = q4.DecodeStack(gemvs, 4)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        st.run(status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check_all(gemvs, host, 4, "two levels back")
