@@ -221,6 +221,9 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     constexpr int WPT = L / 4;
     constexpr int STAGEK = kTileBytes * 8 / BITS;
     constexpr int LANES = STAGEK / 8;
+    // parts of x read at a time when a slot is built (measured: four for int4 codes; the
+    // int8 kernel, tighter on registers, keeps two)
+    constexpr int QB = BITS == 4 ? 4 : 2;
     constexpr int GS = GPS > 0 ? GPS : 1;
     constexpr int FSLOT = slot1_bytes<BITS>();  // B fragments of one tile + format header
     extern __shared__ uint8_t smem_raw[];
@@ -430,20 +433,23 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                         const size_t st4 = (size_t)BE->xstride / 4;
                         const int pm = BE->xpmax;
                         float4 s0 = __ldcg(src), s1 = __ldcg(src + 1);
-                        for (int q0 = 1; q0 < pm; q0 += 2) {
-                            const bool two = q0 + 1 < pm;
-                            const float4 b0 = __ldcg(src + q0 * st4), b1 = __ldcg(src + q0 * st4 + 1);
-                            float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
-                            if (two) {
-                                c0 = __ldcg(src + (q0 + 1) * st4);
-                                c1 = __ldcg(src + (q0 + 1) * st4 + 1);
+                        // QB parts in flight at a time, added in part order
+                        for (int q0 = 1; q0 < pm; q0 += QB) {
+                            float4 b[QB][2];
+#pragma unroll
+                            for (int j = 0; j < QB; ++j) {
+                                b[j][0] = b[j][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                if (q0 + j < pm) {
+                                    b[j][0] = __ldcg(src + (q0 + j) * st4);
+                                    b[j][1] = __ldcg(src + (q0 + j) * st4 + 1);
+                                }
                             }
-                            s0.x += b0.x; s0.y += b0.y; s0.z += b0.z; s0.w += b0.w;
-                            s1.x += b1.x; s1.y += b1.y; s1.z += b1.z; s1.w += b1.w;
-                            if (two) {
-                                s0.x += c0.x; s0.y += c0.y; s0.z += c0.z; s0.w += c0.w;
-                                s1.x += c1.x; s1.y += c1.y; s1.z += c1.z; s1.w += c1.w;
-                            }
+#pragma unroll
+                            for (int j = 0; j < QB; ++j)
+                                if (q0 + j < pm) {
+                                    s0.x += b[j][0].x; s0.y += b[j][0].y; s0.z += b[j][0].z; s0.w += b[j][0].w;
+                                    s1.x += b[j][1].x; s1.y += b[j][1].y; s1.z += b[j][1].z; s1.w += b[j][1].w;
+                                }
                         }
                         v[0] = s0.x; v[1] = s0.y; v[2] = s0.z; v[3] = s0.w;
                         v[4] = s1.x; v[5] = s1.y; v[6] = s1.z; v[7] = s1.w;
