@@ -209,6 +209,22 @@ Q4_DEVINL bool wait_fin(const int *fin_done, const StackLevel *lev, int lo, int 
     return true;
 }
 
+// The output of a split row block's sum (see the consumers' finalize).
+struct FinSrc {
+    const float *parts;
+    float *y;
+    int N, npad, pmax, pad;
+};
+
+// Where the activations of a slot come from (see the consumers' slot build).
+struct SlotSrc {
+    const float *xp;  // non-null: x is the sum of these parts
+    const void *x;    // otherwise x itself
+    int k0, K;        // first k of the stage; K of the GEMV
+    int pm, st4;      // parts; their row stride in float4
+    int i;            // tile (relative to the CTA's first of the level)
+};
+
 // First scale group of k-stage s.
 template <int GPS, int STAGEK>
 Q4_DEVINL int stage_group(int s, int group) {
@@ -236,6 +252,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: a wait of this CTA gave up
     int *finq = flag + 4;  // [warp][2][4] pending sums of split row blocks: {entry, rb, parts, level}
     int *pubq = finq + kConsumers * 8;  // [8] warps arrived at each of the last eight publications
+    SlotSrc *srcq = reinterpret_cast<SlotSrc *>(pubq + 8);  // [warp] its first slot's source
+    FinSrc *fsrc = reinterpret_cast<FinSrc *>(srcq + kConsumers);  // level l - 2's block
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, G = a.G;
@@ -323,17 +341,27 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
         __syncwarp();
         // the sum of split row block f, parts in order, by warps w0..14 (the others are busy
         // building); one release for the block once all of them have written their rows
-        auto finalize = [&](const int *f, int w0) {
+        auto fin_src = [&](const int *f) {
+            const StackEntry *fe = a.ent + f[0];
+            FinSrc r;
+            r.parts = fe->parts;
+            r.y = fe->y;
+            r.N = fe->N;
+            r.npad = fe->npad;
+            r.pmax = fe->pmax;
+            r.pad = 0;
+            return r;
+        };
+        auto finalize = [&](const int *f, const FinSrc fe, int w0) {
             if (warp < w0) return;
             const int nw = kConsumers - w0;
-            const StackEntry *fe = a.ent + f[0];
             const int np = f[2];
-            const size_t st = (size_t)fe->npad;
+            const size_t st = (size_t)fe.npad;
             for (int rr = (warp - w0) * 32 + lane; rr < kSRows; rr += nw * 32) {
                 const int row = f[1] * kSRows + rr;
-                if (row < fe->N) {
+                if (row < fe.N) {
                     // four loads in flight at a time, added in part order
-                    const float *pp = fe->parts + row;
+                    const float *pp = fe.parts + row;
                     float v = 0.f;
                     for (int q0 = 0; q0 < np; q0 += 4) {
                         float pv[4];
@@ -343,8 +371,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                         for (int j = 0; j < 4; ++j)
                             if (q0 + j < np) v = q0 + j == 0 ? pv[0] : v + pv[j];
                     }
-                    if (np < fe->pmax) v += 0.f;  // as the sum over all pmax parts, zeros included
-                    fe->y[row] = v;
+                    if (np < fe.pmax) v += 0.f;  // as the sum over all pmax parts, zeros included
+                    fe.y[row] = v;
                 }
             }
             named_barrier_sync(2, nw * 32);
@@ -369,6 +397,28 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             StackLevel lv;
             Cursor cu;
             if (l < a.L) lv = a.lev[l];
+            // where the x of tile i (relative to u0) comes from: the tables only, so a warp
+            // reads its first slot's before the wait for the previous level
+            auto slot_src = [&](int i) {
+                SlotSrc r;
+                const Cursor bc = cursor_at(a.ent, lv, u0 + i);
+                const StackEntry *BE = a.ent + bc.e;
+                r.xp = XBF16 ? nullptr : BE->xparts;
+                r.x = BE->x;
+                r.k0 = bc.s * STAGEK;
+                r.K = BE->K;
+                r.pm = BE->xpmax;
+                r.st4 = BE->xstride / 4;
+                r.i = i;
+                return r;
+            };
+            // the entry of level l - 2's block, read while the level waits
+            if (has_old && warp == kConsumers - 1 && lane == 0) *fsrc = fin_src(f_old);
+            const bool has_first = n > 0 && warp < min(n, a.ucap);
+            if (has_first) {
+                const SlotSrc f = slot_src(warp);
+                if (lane == 0) srcq[warp] = f;
+            }
             if (n > 0) {
                 cu = cursor_at(a.ent, lv, u0);
                 // the first tile's scale lines, into L1 while this level waits
@@ -397,8 +447,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             const bool now_new = has_new && (l == a.L || n == 0 || lv.needs_final);
             const int w_free = (l == a.L || n == 0 || lv.needs_final) ? 0 : min(kConsumers, min(n, a.ucap));
             if (w_free < kConsumers) {
-                if (has_old) finalize(f_old, w_free);
-                if (now_new) finalize(f_new, w_free);
+                if (has_old) finalize(f_old, *fsrc, w_free);
+                if (now_new) finalize(f_new, fin_src(f_new), w_free);
             }
             if (lane == 0) {
                 if (has_old && w_free < kConsumers) f_old[0] = -1;
@@ -415,24 +465,23 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             // at a time: exact integer digits or bf16 pieces, decided per tile
             auto build = [&](int i0, int i1) {
                 for (int i = i0 + warp; i < i1; i += kConsumers) {
-                    const Cursor bc = cursor_at(a.ent, lv, u0 + i);
-                    const StackEntry *BE = a.ent + bc.e;
+                    const SlotSrc src = i0 == 0 && i == warp ? srcq[warp] : slot_src(i);
                     uint8_t *bs = bbuf + (size_t)(i - i0) * FSLOT;
-                    const float *xp = XBF16 ? nullptr : BE->xparts;
+                    const float *xp = src.xp;
                     if (!xp) {
-                        build_slot1<BITS, L, XBF16, true>(bs, BE->x, bc.s * STAGEK, BE->K, a.P, lane);
+                        build_slot1<BITS, L, XBF16, true>(bs, src.x, src.k0, src.K, a.P, lane);
                         continue;
                     }
                     // x = the sum of the producing GEMV's parts of these rows, in part order
                     float v[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) v[q] = 0.f;
-                    const int k = bc.s * STAGEK + 8 * lane;
-                    if (lane < LANES && k < BE->K) {
-                        const float4 *src = reinterpret_cast<const float4 *>(xp + k);
-                        const size_t st4 = (size_t)BE->xstride / 4;
-                        const int pm = BE->xpmax;
-                        float4 s0 = __ldcg(src), s1 = __ldcg(src + 1);
+                    const int k = src.k0 + 8 * lane;
+                    if (lane < LANES && k < src.K) {
+                        const float4 *xq = reinterpret_cast<const float4 *>(xp + k);
+                        const size_t st4 = (size_t)src.st4;
+                        const int pm = src.pm;
+                        float4 s0 = __ldcg(xq), s1 = __ldcg(xq + 1);
                         // QB parts in flight at a time, added in part order
                         for (int q0 = 1; q0 < pm; q0 += QB) {
                             float4 b[QB][2];
@@ -440,8 +489,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                             for (int j = 0; j < QB; ++j) {
                                 b[j][0] = b[j][1] = make_float4(0.f, 0.f, 0.f, 0.f);
                                 if (q0 + j < pm) {
-                                    b[j][0] = __ldcg(src + (q0 + j) * st4);
-                                    b[j][1] = __ldcg(src + (q0 + j) * st4 + 1);
+                                    b[j][0] = __ldcg(xq + (q0 + j) * st4);
+                                    b[j][1] = __ldcg(xq + (q0 + j) * st4 + 1);
                                 }
                             }
 #pragma unroll
@@ -460,7 +509,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             int chunk_lo = 0, chunk_hi = min(n, a.ucap);
             build(0, chunk_hi);
             if (has_old && w_free == kConsumers) {  // every warp built: the sum comes after
-                finalize(f_old, 0);
+                finalize(f_old, *fsrc, 0);
                 if (lane == 0) f_old[0] = -1;
                 __syncwarp();
             }
@@ -757,7 +806,8 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
     const size_t fslot = bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>();  // B fragments + header of a tile
     const int kRing = ring_of(lo.gps);
     const size_t budget = (size_t)smem_budget_of(lo.gps);
-    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4 + 8 * 4;
+    const size_t fixed = 1024 + (size_t)kRing * kSTile + 2 * kRing * 8 + 16 + kConsumers * 8 * 4 + 8 * 4 +
+                         kConsumers * sizeof(SlotSrc) + sizeof(FinSrc);
     if (fixed + fslot > budget) return Q4_ERR_UNSUPPORTED;
     int ucap = (int)((budget - fixed) / fslot);
     if (ucap > ucap_max_of(lo.gps)) ucap = ucap_max_of(lo.gps);
