@@ -19,7 +19,9 @@
 //     the current level ends.
 //   * Fifteen consumer warps (16 rows of each tile apiece) wait (bounded, on a device
 //     counter) until every part of the previous level is published, build the exact
-//     digits or bf16 pieces of x for their tiles, and multiply.
+//     digits or bf16 pieces of x for their tiles, and multiply. What a slot build needs
+//     from the tables (which GEMV, where its x or parts are) is read before the wait, so
+//     after it only the loads of x remain.
 //   * A row block whose k-stages fall to several CTAs ends as several parts, one per
 //     CTA, kept in a [parts][rows] matrix per GEMV; a part is published with one release
 //     increment of the level's counter, without waiting for the other parts. Nobody
