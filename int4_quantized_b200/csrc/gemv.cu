@@ -161,8 +161,10 @@ __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
 // otherwise the pieces come from gemv_prep through a second ring. GPS: groups per stage
 // when they divide it, 0 when the stage lies inside one group, -1 for any other group
 // size (tracked segment by segment at run time).
-template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB>
-__global__ void __launch_bounds__(kThreads) __maxnreg__(NB >= 3 ? 160 : 96)
+// WIDE: one CTA per SM, so the registers of two (the plan's choice for few piece columns
+// when the grid stays full; see plan_gemv)
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB, bool WIDE>
+__global__ void __launch_bounds__(kThreads) __maxnreg__(NB >= 3 || WIDE ? 160 : 96)
 gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     constexpr int SPS = kTileBytes / (4 * L);          // segments per stage
     constexpr int KTI = BITS == 4 ? L / 2 : L / 4;     // MMAs per segment
@@ -564,7 +566,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
 // early: the weights are static, so the call's first grid may start (and the stream
 // kernel read payload and scales) while the previous kernel on the stream still runs.
 // Every read of x, and every write, still waits for that kernel to finish.
-template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB = false>
+template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB = false, bool WIDE = false>
 cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
                          bool early, cudaStream_t st) {
     cudaError_t err;
@@ -585,7 +587,7 @@ cudaError_t launch_typed(const GemvPlan &pl, const GemvArgs &a, const CUtensorMa
                      : cudaLaunchKernelEx(&pc, gemv_prep<BITS, L, false, HYB>, a);
         if (err != cudaSuccess) return err;
     }
-    auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16, HYB>;
+    auto kern = gemv_stream<BITS, L, NB, GPS, INK, XBF16, HYB, WIDE>;
     const size_t smem = pl.smem_bytes;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
@@ -626,8 +628,14 @@ cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorM
                                     pl, a, tm, false, early, st);                                \
         }                                                                                        \
         switch (pl.NB) {                                                                         \
-            case 1: return launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, early, st); \
-            case 2: return launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, early, st); \
+            case 1:                                                                              \
+                return pl.ctas_per_sm == 1                                                       \
+                           ? launch_typed<B, LL, 1, G, false, false, false, true>(pl, a, tm, x_bf16, early, st) \
+                           : launch_typed<B, LL, 1, G, false, false>(pl, a, tm, x_bf16, early, st);    \
+            case 2:                                                                              \
+                return pl.ctas_per_sm == 1                                                       \
+                           ? launch_typed<B, LL, 2, G, false, false, false, true>(pl, a, tm, x_bf16, early, st) \
+                           : launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, early, st);    \
             case 3: return launch_typed<B, LL, 3, G, false, false>(pl, a, tm, x_bf16, early, st); \
             case 4: return launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, early, st); \
             default: return launch_typed<B, LL, 6, G, false, false>(pl, a, tm, x_bf16, early, st); \
@@ -716,6 +724,12 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, bool x_
     p.n_eb = (p.stages_total + p.ebs - 1) / p.ebs;
     // many piece columns need a deep ring of large slots: one CTA per SM
     p.ctas_per_sm = p.NB >= 3 ? 1 : 2;
+    // one or two column blocks of several fp32 rows of x: one CTA per SM with the registers
+    // of two (no spills) when the K split over a cluster can still be 2 or more; else two
+    // per SM keep more CTAs in flight (4096x4096, M = 4: 13.5 -> 8.6 us; 11008x4096, M = 4:
+    // 15.5 us with two per SM, 18.7 us with one)
+    const int64_t blocks0 = (int64_t)p.clusters * p.nmc;
+    if (p.NB <= 2 && M > 1 && !x_bf16 && blocks0 > 0 && sms / blocks0 >= 2) p.ctas_per_sm = 1;
     const size_t budget = p.ctas_per_sm == 2 ? kSmemBudget2 : kSmemBudget1;
     // split K over a cluster so that the grid is one wave
     const int64_t slots = (int64_t)sms * p.ctas_per_sm;
