@@ -31,7 +31,9 @@
 //     the CTA holding its last part, as the same sum, so y and what the next level read
 //     are the same numbers; it does so at the start of the level after next, on the warps
 //     that have no slot to build while the others build (at the next start, before the
-//     build, if the next level reads that y directly). A level waits for the sums of three
+//     build, if the next level reads that y directly). Those warps post their release as a
+//     ticket in shared memory; the producer warp takes it between two loads and makes the
+//     GPU-scope release, so no consumer waits for the rows' stores to land. A level waits for the sums of three
 //     levels back (the parts buffers rotate over three levels) and of every earlier level
 //     whose y it reads directly.
 //   * Counters return to zero at the end of every launch (the last CTA to finish resets
@@ -129,6 +131,11 @@ Q4_DEVINL int ld_acquire(const int *p) {
 // __syncwarp() before each call orders the other lanes' writes first).
 Q4_DEVINL void red_release_add(int *p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+Q4_DEVINL int atom_exch_acq_rel_cta_shared(int *p, int v) {
+    int old;
+    asm volatile("atom.exch.acq_rel.cta.shared.b32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
 }
 Q4_DEVINL int atom_acq_rel_cta_shared_add(int *p, int v) {
     int old;
@@ -252,6 +259,13 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     uint64_t *full = reinterpret_cast<uint64_t *>(bbuf + (size_t)a.ucap * FSLOT);
     uint64_t *empty = full + kRing;
     int *flag = reinterpret_cast<int *>(empty + kRing);  // [0]: a wait of this CTA gave up
+    int *ticket = flag + 2;  // split-block sums written and not yet released: their level + 1
+    // the GPU-scope release of a posted ticket (whoever takes it: the producer between its
+    // loads, warp 0 before it waits, thread 0 at the end)
+    auto take_ticket = [&]() {
+        const int tk = atom_exch_acq_rel_cta_shared(ticket, 0);
+        if (tk) red_release_add(a.fin_done + tk - 1, 1);
+    };
     int *finq = flag + 4;  // [warp][2][4] pending sums of split row blocks: {entry, rb, parts, level}
     int *pubq = finq + kConsumers * 8;  // [8] warps arrived at each of the last eight publications
     SlotSrc *srcq = reinterpret_cast<SlotSrc *>(pubq + 8);  // [warp] its first slot's source
@@ -265,6 +279,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             mbar_init(empty + i, kConsumers);
         }
         flag[0] = 0;
+        flag[2] = 0;  // a posted release of split-block sums: its level + 1, or 0
         for (int i = 0; i < 8; ++i) pubq[i] = 0;
         fence_barrier_init();
     }
@@ -294,6 +309,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                     R = E->R;
                     tmap_acquire(&E->tm);
                 }
+                if (lane == 0) take_ticket();
                 if (round > 0 && !timed_out) timed_out = !mbar_wait(empty + slot, (uint32_t)((round - 1) & 1), a.wait_ns);
                 if (lane == 0 && !timed_out) {
                     mbar_arrive_expect_tx(full + slot, kSTile);
@@ -354,7 +370,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             r.pad = 0;
             return r;
         };
-        auto finalize = [&](const int *f, const FinSrc fe, int w0) {
+        auto finalize = [&](const int *f, const FinSrc fe, int w0, bool post) {
             if (warp < w0) return;
             const int nw = kConsumers - w0;
             const int np = f[2];
@@ -362,15 +378,15 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             for (int rr = (warp - w0) * 32 + lane; rr < kSRows; rr += nw * 32) {
                 const int row = f[1] * kSRows + rr;
                 if (row < fe.N) {
-                    // four loads in flight at a time, added in part order
+                    // twelve loads in flight at a time, added in part order
                     const float *pp = fe.parts + row;
                     float v = 0.f;
-                    for (int q0 = 0; q0 < np; q0 += 4) {
-                        float pv[4];
+                    for (int q0 = 0; q0 < np; q0 += 12) {
+                        float pv[12];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) pv[j] = q0 + j < np ? __ldcg(pp + (q0 + j) * st) : 0.f;
+                        for (int j = 0; j < 12; ++j) pv[j] = q0 + j < np ? __ldcg(pp + (q0 + j) * st) : 0.f;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 12; ++j)
                             if (q0 + j < np) v = q0 + j == 0 ? pv[0] : v + pv[j];
                     }
                     if (np < fe.pmax) v += 0.f;  // as the sum over all pmax parts, zeros included
@@ -379,8 +395,16 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             }
             named_barrier_sync(2, nw * 32);
             if (warp == w0 && lane == 0) {
-                __threadfence();
-                red_release_add(a.fin_done + f[3], 1);
+                if (post) {
+                    // a CTA-scope release of the rows to whoever takes the ticket, so these
+                    // warps do not wait for their stores to land (an older ticket still
+                    // posted is released here)
+                    const int old = atom_exch_acq_rel_cta_shared(ticket, f[3] + 1);
+                    if (old) red_release_add(a.fin_done + old - 1, 1);
+                } else {
+                    __threadfence();
+                    red_release_add(a.fin_done + f[3], 1);
+                }
             }
         };
         for (int l = 0; l <= a.L; ++l) {
@@ -435,7 +459,10 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 // level has published its rows, and the levels this one needs have their sums
                 if (warp == 0 && !timed_out) {
                     bool ok = true;
-                    if (lane == 0) ok = wait_counter(a.parts_done + (l - 1), a.lev[l - 1].parts_target, a.wait_ns);
+                    if (lane == 0) {
+                        take_ticket();  // never wait on sums of this CTA's own not yet released
+                        ok = wait_counter(a.parts_done + (l - 1), a.lev[l - 1].parts_target, a.wait_ns);
+                    }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (ok && l < a.L) ok = wait_fin(a.fin_done, a.lev, lv.fin_lo, lv.fin_hi, a.wait_ns, lane);
                     timed_out = !ok;
@@ -449,8 +476,8 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             const bool now_new = has_new && (l == a.L || n == 0 || lv.needs_final);
             const int w_free = (l == a.L || n == 0 || lv.needs_final) ? 0 : min(kConsumers, min(n, a.ucap));
             if (w_free < kConsumers) {
-                if (has_old) finalize(f_old, *fsrc, w_free);
-                if (now_new) finalize(f_new, fin_src(f_new), w_free);
+                if (has_old) finalize(f_old, *fsrc, w_free, l < a.L && n > 0);
+                if (now_new) finalize(f_new, fin_src(f_new), w_free, false);
             }
             if (lane == 0) {
                 if (has_old && w_free < kConsumers) f_old[0] = -1;
@@ -511,7 +538,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
             int chunk_lo = 0, chunk_hi = min(n, a.ucap);
             build(0, chunk_hi);
             if (has_old && w_free == kConsumers) {  // every warp built: the sum comes after
-                finalize(f_old, *fsrc, 0);
+                finalize(f_old, *fsrc, 0, true);
                 if (lane == 0) f_old[0] = -1;
                 __syncwarp();
             }
@@ -640,6 +667,7 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
     if (timed_out) flag[0] = 1;
     __syncthreads();
     if (threadIdx.x == 0) {
+        take_ticket();
         if (flag[0] && a.status) atomicOr(a.status, Q4_STATUS_TIMEOUT);
         __threadfence();
         const int old = atomicAdd(a.finished, 1);
