@@ -459,12 +459,13 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 // level has published its rows, and the levels this one needs have their sums
                 if (warp == 0 && !timed_out) {
                     bool ok = true;
-                    if (lane == 0) {
-                        take_ticket();  // never wait on sums of this CTA's own not yet released
-                        ok = wait_counter(a.parts_done + (l - 1), a.lev[l - 1].parts_target, a.wait_ns);
-                    }
+                    if (lane == 0) take_ticket();  // never wait on sums of this CTA's own not yet released
+                    __syncwarp();
+                    // the sums first: they are older and usually long in y, so their check
+                    // is over before the previous level ends
+                    if (l < a.L) ok = wait_fin(a.fin_done, a.lev, lv.fin_lo, lv.fin_hi, a.wait_ns, lane);
+                    if (ok && lane == 0) ok = wait_counter(a.parts_done + (l - 1), a.lev[l - 1].parts_target, a.wait_ns);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (ok && l < a.L) ok = wait_fin(a.fin_done, a.lev, lv.fin_lo, lv.fin_hi, a.wait_ns, lane);
                     timed_out = !ok;
                 }
                 named_barrier_sync(1, kConsumerThreads);
