@@ -577,10 +577,24 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                     const int ng = min(GS, spr - gbase);
                     const float *sp0 = scales + (size_t)min(cu.rb * kSRows + pr, N - 1) * spr + gbase;
                     const float *sp1 = scales + (size_t)min(cu.rb * kSRows + pr + 8, N - 1) * spr + gbase;
+                    // four groups a stage (g64 int4): one vector load per row when they are
+                    // whole and aligned (measured: with two groups the vector form makes the
+                    // kernel spill)
+                    const bool vec = GS == 4 && ng == GS &&
+                                     ((reinterpret_cast<uintptr_t>(sp0) | reinterpret_cast<uintptr_t>(sp1)) & 15u) == 0;
+                    if (vec) {
+                        if constexpr (GS == 4) {
+                            const float4 v0 = __ldg(reinterpret_cast<const float4 *>(sp0));
+                            const float4 v1 = __ldg(reinterpret_cast<const float4 *>(sp1));
+                            s0r[0] = v0.x; s0r[1] = v0.y; s0r[2] = v0.z; s0r[3] = v0.w;
+                            s1r[0] = v1.x; s1r[1] = v1.y; s1r[2] = v1.z; s1r[3] = v1.w;
+                        }
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < GS; ++q) {
-                        s0r[q] = q < ng ? __ldg(sp0 + q) : 0.f;
-                        s1r[q] = q < ng ? __ldg(sp1 + q) : 0.f;
+                        for (int q = 0; q < GS; ++q) {
+                            s0r[q] = q < ng ? __ldg(sp0 + q) : 0.f;
+                            s1r[q] = q < ng ? __ldg(sp1 + q) : 0.f;
+                        }
                     }
                 }
                 if (!timed_out) timed_out = !mbar_wait(full + slot, (uint32_t)(round & 1), a.wait_ns);
