@@ -161,10 +161,10 @@ __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
 // otherwise the pieces come from gemv_prep through a second ring. GPS: groups per stage
 // when they divide it, 0 when the stage lies inside one group, -1 for any other group
 // size (tracked segment by segment at run time).
-// WIDE: one CTA per SM, so the registers of two (the plan's choice for few piece columns
-// when the grid stays full; see plan_gemv)
+// WIDE: one CTA per SM, so the registers of two (the plan's choice for up to four column
+// blocks when the grid stays full; see gemv_plan)
 template <int BITS, int L, int NB, int GPS, bool INK, bool XBF16, bool HYB, bool WIDE>
-__global__ void __launch_bounds__(kThreads) __maxnreg__(NB >= 3 || WIDE ? 160 : 96)
+__global__ void __launch_bounds__(kThreads) __maxnreg__(NB >= 5 || WIDE ? 160 : 96)
 gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     constexpr int SPS = kTileBytes / (4 * L);          // segments per stage
     constexpr int KTI = BITS == 4 ? L / 2 : L / 4;     // MMAs per segment
@@ -636,8 +636,14 @@ cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorM
                 return pl.ctas_per_sm == 1                                                       \
                            ? launch_typed<B, LL, 2, G, false, false, false, true>(pl, a, tm, x_bf16, early, st) \
                            : launch_typed<B, LL, 2, G, false, false>(pl, a, tm, x_bf16, early, st);    \
-            case 3: return launch_typed<B, LL, 3, G, false, false>(pl, a, tm, x_bf16, early, st); \
-            case 4: return launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, early, st); \
+            case 3:                                                                              \
+                return pl.ctas_per_sm == 1                                                       \
+                           ? launch_typed<B, LL, 3, G, false, false, false, true>(pl, a, tm, x_bf16, early, st) \
+                           : launch_typed<B, LL, 3, G, false, false>(pl, a, tm, x_bf16, early, st);    \
+            case 4:                                                                              \
+                return pl.ctas_per_sm == 1                                                       \
+                           ? launch_typed<B, LL, 4, G, false, false, false, true>(pl, a, tm, x_bf16, early, st) \
+                           : launch_typed<B, LL, 4, G, false, false>(pl, a, tm, x_bf16, early, st);    \
             default: return launch_typed<B, LL, 6, G, false, false>(pl, a, tm, x_bf16, early, st); \
         }                                                                                        \
     }
@@ -724,12 +730,13 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, bool x_
     p.n_eb = (p.stages_total + p.ebs - 1) / p.ebs;
     // many piece columns need a deep ring of large slots: one CTA per SM
     p.ctas_per_sm = p.NB >= 3 ? 1 : 2;
-    // one or two column blocks of several fp32 rows of x: one CTA per SM with the registers
-    // of two (no spills) when the K split over a cluster can still be 2 or more; else two
-    // per SM keep more CTAs in flight (4096x4096, M = 4: 13.5 -> 8.6 us; 11008x4096, M = 4:
-    // 15.5 us with two per SM, 18.7 us with one)
+    // fp32 rows of x in one to four column blocks: one CTA per SM (the registers of two)
+    // when the K split over a cluster can still be 2 or more, else two per SM at 96
+    // registers, which keeps more CTAs in flight (measured, int4 g128 with static weights:
+    // 4096x4096 M = 4 13.5 -> 8.6 us with one per SM; 11008x4096 M = 4 15.5 us with two
+    // per SM, 18.7 with one; M = 8 23.7 -> 18.1 us with two)
     const int64_t blocks0 = (int64_t)p.clusters * p.nmc;
-    if (p.NB <= 2 && M > 1 && !x_bf16 && blocks0 > 0 && sms / blocks0 >= 2) p.ctas_per_sm = 1;
+    if (p.NB <= 4 && M > 1 && !x_bf16 && blocks0 > 0) p.ctas_per_sm = sms / blocks0 >= 2 ? 1 : 2;
     const size_t budget = p.ctas_per_sm == 2 ? kSmemBudget2 : kSmemBudget1;
     // split K over a cluster so that the grid is one wave
     const int64_t slots = (int64_t)sms * p.ctas_per_sm;

@@ -88,7 +88,8 @@ def test_mid_config_full(q4, M):
 
 
 @pytest.mark.parametrize("idx", [0, 4, 6])   # q (4096x4096), gate (11008x4096), down (4096x11008)
-@pytest.mark.parametrize("M", [1, 4, 16])
+# M = 4, 8, 10: one to four column blocks, one CTA per SM on 4096 rows and two on 11008
+@pytest.mark.parametrize("M", [1, 4, 8, 10, 16])
 def test_llama7b_sampled(q4, idx, M):
     wl = workloads.WORKLOADS["llama7b"]
     m = wl.matrices[idx]
