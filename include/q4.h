@@ -122,7 +122,9 @@ Q4_API q4_status qdequant(const uint8_t *payload, const float *scales, int64_t r
  * into tensor-core fragments (exact bf16 pieces, 3 per fp32 activation, in MMA order;
  * for one row of x, per 128-byte stage either those pieces or exact 40-bit fixed-point
  * digits, 2064 bytes per int4 stage and 1040 per int8 stage). One row of x needs none (0)
- * when each CTA's share of K, at most 4096, is built on chip. Groups of whole rows
+ * when each CTA's share of K, at most 4096, is built on chip; so do two to four fp32 rows
+ * when, in addition, the plan runs one CTA per SM (N up to 74 x 128 rows, as planned for
+ * 148 SMs) and their pieces fit in its shared memory. Groups of whole rows
  * (group a multiple of K) add N floats, rounded up to 256 bytes, at the start: their
  * scales spread to one per row. The any-group path needs none (0). Same arguments as
  * qgemm. Returns 0 for arguments qgemm rejects. Depends only on the arguments, not on

@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(256) gemv_prep(const GemvArgs a) {
     }
 }
 
-// INK: one row of x whose pieces the consumers build in shared memory (no workspace);
-// otherwise the pieces come from gemv_prep through a second ring. GPS: groups per stage
+// INK: the pieces of one row of x, or of two to four fp32 rows (one or two column blocks),
+// are built by the consumers in shared memory (no workspace); otherwise they come from
+// gemv_prep through a second ring. GPS: groups per stage
 // when they divide it, 0 when the stage lies inside one group, -1 for any other group
 // size (tracked segment by segment at run time).
 // WIDE: one CTA per SM, so the registers of two (the plan's choice for up to four column
@@ -172,8 +173,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
     constexpr int WPT = L / 4;
     constexpr int STAGEK = kTileBytes * 8 / BITS;
     constexpr bool PAIRED = NB <= 2;
-    constexpr int LW = INK ? 16 : 32;  // piece lanes stored per (MMA, n8 block), workspace: a.lw
-    static_assert(!INK || NB == 1, "on-chip pieces cover one row of x");
+    static_assert(!INK || NB <= 2, "on-chip pieces cover at most two column blocks");
     static_assert(!HYB || (NB == 1 && GPS >= 0), "one row of x, regular groups");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -336,27 +336,27 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                                                   a.K, a.P, lane);
             named_barrier_sync(1, kConsumerThreads);
         } else if constexpr (INK) {
-            // pieces of this CTA's K range of the single activation row, built while the
-            // first payload tiles are in flight; column 3 (and the 16 lanes above, which
-            // repeat these) is zero
+            // pieces of this CTA's K range of the rows of x, built while the first payload
+            // tiles are in flight (one item, 8 k of one row, per thread at a time, as in
+            // gemv_prep); columns past the rows (and the lanes past the stored width, which
+            // repeat these) are zero
             const int k_lo = st_lo * STAGEK, k_hi = min(st_hi * STAGEK, a.K);
             const int nu = max(k_hi - k_lo, 0) / 8;
-            constexpr int R = kInkMaxK / 8 / kConsumerThreads;  // units per thread (2)
+            const int ncols = stored_cols(NB, a.lw);
+            const int vrows = (ncols + a.P - 1) / a.P;
             uint2 *fbase = reinterpret_cast<uint2 *>(fslots);
+            for (int it = ct; it < nu * vrows; it += kConsumerThreads) {
+                const int vm = it / nu, u = it - vm * nu;
+                float v[8];
+                if (vm < a.M) {
+                    load_x8<XBF16>(a.x, (int64_t)vm * a.K + k_lo + 8 * u, v);
+                } else {
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int u = ct + kConsumerThreads * r;
-                if (u < nu) {
-                    float v[8];
-                    load_x8<XBF16>(a.x, (int64_t)k_lo + 8 * u, v);
-                    const int ls = (8 * u) / STAGEK;  // local stage
-                    float z[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) z[q] = 0.f;
-                    uint2 *st = fbase + (size_t)ls * (a.fslot_bytes / 8);
-                    frag_unit<BITS, L>(st, 8 * u - ls * STAGEK, 0, v, a.P, 4, 1, LW, true);
-                    for (int vm = 1; vm * a.P < 4; ++vm) frag_unit<BITS, L>(st, 8 * u - ls * STAGEK, vm, z, a.P, 4, 1, LW, true);
+                    for (int q = 0; q < 8; ++q) v[q] = 0.f;
                 }
+                const int ls = (8 * u) / STAGEK;  // local stage
+                frag_unit<BITS, L>(fbase + (size_t)ls * (a.fslot_bytes / 8), 8 * u - ls * STAGEK, vm, v, a.P, ncols,
+                                   NB, a.lw, a.paired != 0);
             }
             named_barrier_sync(1, kConsumerThreads);
         }
@@ -367,7 +367,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
             const int off = sl * 4 * L + t * L;
             aoff[sl] = pr * kTileBytes + (((off >> 4) ^ (pr & 7)) << 4) + (off & 15);
         }
-        const int lwr = INK ? LW : a.lw;
+        const int lwr = a.lw;
         const int fl = lane & (lwr - 1);  // lanes past the stored width repeat lanes (their columns are unused)
         float ys0 = 0.f, ys1 = 0.f;  // one row of x: this lane's share of rows pr and pr + 8
         float cacc[NB][4], acc[NB][4];
@@ -446,7 +446,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
                 const int qb = (GPS > 0 ? s * GPS : (s * SPS) / a.spg) - gA;  // first group, in the k-block
                 const float *s0p = sb + pr * kSG + qb, *s1p = s0p + 8 * kSG;
                 const uint8_t *frl = fr + fl * (PAIRED ? 16 : 8);
-                if (INK || a.lw == 16) {
+                if (lwr == 16) {
                     if (nsl == SPS)
                         stage_fixed<BITS, L, NB, 16, GPS, true>(A0, A1, frl, s0p, s1p, nsl, acc);
                     else
@@ -469,7 +469,7 @@ gemv_stream(const GemvArgs a, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb) {
                             uint32_t b0, b1;
-                            if (INK || lwr == 16)
+                            if (lwr == 16)
                                 load_b<NB, 16, PAIRED>(frl, i, nb, bq, b0, b1);
                             else
                                 load_b<NB, 32, PAIRED>(frl, i, nb, bq, b0, b1);
@@ -615,9 +615,13 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 cudaError_t dispatch_gemv(const GemvPlan &pl, const GemvArgs &a, const CUtensorMap &tm, bool x_bf16,
                           bool early, cudaStream_t st) {
 #define Q4_INK(B, LL, G)                                                                         \
-    if (pl.bits == B && pl.L == LL && pl.gps == G)                                               \
+    if (pl.bits == B && pl.L == LL && pl.gps == G) {                                             \
+        if (a.M > 1)                                                                             \
+            return pl.NB == 2 ? launch_typed<B, LL, 2, G, true, false, false, true>(pl, a, tm, false, early, st) \
+                              : launch_typed<B, LL, 1, G, true, false, false, true>(pl, a, tm, false, early, st); \
         return x_bf16 ? launch_typed<B, LL, 1, G, true, true, (G >= 0)>(pl, a, tm, true, early, st) \
-                      : launch_typed<B, LL, 1, G, true, false, (G >= 0)>(pl, a, tm, false, early, st);
+                      : launch_typed<B, LL, 1, G, true, false, (G >= 0)>(pl, a, tm, false, early, st); \
+    }
 #define Q4_STAGED(B, LL, G)                                                                      \
     if (pl.bits == B && pl.L == LL && pl.gps == G) {                                             \
         if (pl.hyb) {                                                                            \
@@ -754,6 +758,12 @@ bool gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int64_t group, bool x_
     p.hyb = M == 1 && p.gps >= 0;
     p.fslot_bytes = p.hyb ? (bits == 4 ? slot1_bytes<4>() : slot1_bytes<8>()) : kts * p.NB * p.lw * 8;
     const size_t fixed = 1024 + 2 * (size_t)kRowsPerCta * kSG * 4 + (4 * kMaxStages + 4) * 8;
+    // two to four fp32 rows at one CTA per SM: their pieces are built on chip too when the
+    // CTA's K range and its slots fit (no gemv_prep launch, no workspace round trip)
+    if (!p.ink && M > 1 && M <= 4 && !x_bf16 && p.NB <= 2 && p.ctas_per_sm == 1 &&
+        (int64_t)p.stages_per_cta * stagek <= kInkMaxK &&
+        budget >= fixed + (size_t)p.stages_per_cta * p.fslot_bytes + 2 * (size_t)kPayloadBytes)
+        p.ink = true;
     int nr;
     if (p.ink) {
         const size_t frag = (size_t)p.stages_per_cta * p.fslot_bytes;

@@ -91,8 +91,14 @@ def test_qgemm_workspace_rules(q4):
     lib = q4.lib()
     need = lib.q4_qgemm_workspace_bytes(8, 4096, 4096, 4, 128, 0)
     assert need > 0 and need % 256 == 0
-    # one row of x needs less fragment space than four
-    assert lib.q4_qgemm_workspace_bytes(1, 4096, 4096, 4, 128, 0) < lib.q4_qgemm_workspace_bytes(4, 4096, 4096, 4, 128, 0)
+    # one row of x needs less fragment space than four (11008 rows: two CTAs per SM, the
+    # pieces of four rows come from the workspace); 4096 rows: up to four fp32 rows are
+    # built on chip, one bf16 row too
+    assert lib.q4_qgemm_workspace_bytes(1, 11008, 4096, 4, 128, 0) < lib.q4_qgemm_workspace_bytes(4, 11008, 4096, 4, 128, 0)
+    for m in (1, 2, 3, 4):
+        assert lib.q4_qgemm_workspace_bytes(m, 4096, 4096, 4, 128, 0) == 0
+    assert lib.q4_qgemm_workspace_bytes(5, 4096, 4096, 4, 128, 0) > 0
+    assert lib.q4_qgemm_workspace_bytes(2, 4096, 4096, 4, 128, 1) > 0  # bf16 rows: from the workspace
     ok = ctypes.c_void_p(0x100000)
     assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, None, None) == 5
     assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need - 1, None, None) == 5
