@@ -89,20 +89,20 @@ def test_qgemm_validation(q4, M, N, K, bits, group, xt, expect):
 
 def test_qgemm_workspace_rules(q4):
     lib = q4.lib()
-    need = lib.q4_qgemm_workspace_bytes(8, 4096, 4096, 4, 128, 0)
+    # 11008 rows: two CTAs per SM, so the pieces of several rows come from the workspace
+    need = lib.q4_qgemm_workspace_bytes(8, 11008, 4096, 4, 128, 0)
     assert need > 0 and need % 256 == 0
-    # one row of x needs less fragment space than four (11008 rows: two CTAs per SM, the
-    # pieces of four rows come from the workspace); 4096 rows: up to four fp32 rows are
-    # built on chip, one bf16 row too
+    # one row of x needs less fragment space than four
     assert lib.q4_qgemm_workspace_bytes(1, 11008, 4096, 4, 128, 0) < lib.q4_qgemm_workspace_bytes(4, 11008, 4096, 4, 128, 0)
+    # 4096 rows, one CTA per SM: up to four fp32 rows (and one bf16 row) are built on chip
     for m in (1, 2, 3, 4):
         assert lib.q4_qgemm_workspace_bytes(m, 4096, 4096, 4, 128, 0) == 0
     assert lib.q4_qgemm_workspace_bytes(5, 4096, 4096, 4, 128, 0) > 0
     assert lib.q4_qgemm_workspace_bytes(2, 4096, 4096, 4, 128, 1) > 0  # bf16 rows: from the workspace
     ok = ctypes.c_void_p(0x100000)
-    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, None, None) == 5
-    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need - 1, None, None) == 5
-    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ctypes.c_void_p(0x100010), need, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 11008, 4096, 4, 128, FAKE, None, need, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 11008, 4096, 4, 128, FAKE, ok, need - 1, None, None) == 5
+    assert lib.qgemm(FAKE, 0, 8, FAKE, FAKE, 11008, 4096, 4, 128, FAKE, ctypes.c_void_p(0x100010), need, None, None) == 5
     # misaligned payload / x are reported before anything is enqueued
     assert lib.qgemm(FAKE, 0, 8, ctypes.c_void_p(0x100001), FAKE, 4096, 4096, 4, 128, FAKE, ok, need, None, None) == 2
     assert lib.qgemm(ctypes.c_void_p(0x100004), 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need, None, None) == 2
@@ -114,14 +114,14 @@ def test_qgemm_workspace_rules(q4):
 def test_qgemm_ex_flags_and_limits(q4):
     lib = q4.lib()
     ok = ctypes.c_void_p(0x100000)
-    need = lib.q4_qgemm_workspace_bytes(8, 4096, 4096, 4, 128, 0)
+    need = lib.q4_qgemm_workspace_bytes(8, 11008, 4096, 4, 128, 0)  # two CTAs per SM: a workspace
     # unknown flag bits are refused before anything else is looked at
     for flags in (2, 4, 0x80000000):
         assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, ok, need, flags, None, None) == 1
     # with the static-weights flag the argument rules are those of qgemm
     assert lib.qgemm_ex(FAKE, 0, 65535 * 16 + 1, FAKE, FAKE, 64, 128, 4, 128, FAKE, None, 0, 1, None, None) == 2
     assert lib.qgemm_ex(FAKE, 0, 1, FAKE, FAKE, 64, 128, 4, 5, FAKE, None, 0, 1, None, None) == 1
-    assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 4096, 4096, 4, 128, FAKE, None, need, 1, None, None) == 5
+    assert lib.qgemm_ex(FAKE, 0, 8, FAKE, FAKE, 11008, 4096, 4, 128, FAKE, None, need, 1, None, None) == 5
     assert lib.qgemm_ex(None, 0, 0, None, None, 4096, 4096, 4, 128, None, None, 0, 1, None, None) == 0
     # rows of x: at most 65535 chunks of 16
     assert q4.qgemm_workspace_bytes(65535 * 16, 256, 1024, 4, 128) > 0
