@@ -13,6 +13,9 @@
 //   * The weight tiles (240 rows x 128 bytes) of a level are numbered GEMV by GEMV, row
 //     block by row block, k-stage by k-stage, and each of the G resident CTAs takes one
 //     contiguous G-th of them (an even split of the level's bytes, whatever its shapes).
+//     Where a level has few row blocks, each row block is split over CTAs of its own
+//     instead, when that keeps the longest range as short: then no range spans two row
+//     blocks, and a row block has fewer parts.
 //   * A producer warp per CTA streams the CTA's tiles of every level, in order, through
 //     one TMA ring, and asks L2 for the scales each stretch of tiles will need. It never
 //     waits for a level: the weights are static, so the next level's tiles arrive while
@@ -905,6 +908,26 @@ q4_status q4_stack_prepare(const q4_stack_gemv *gemvs, int32_t count, int bits, 
         int *us = ustart.data() + (size_t)l * (grid + 1);
         for (int cc = 0; cc <= grid; ++cc)
             us[cc] = lv.U < grid ? (int)std::min<int64_t>(cc, lv.U) : (int)(lv.U * cc / grid);
+        // where row blocks are few: each row block split over its own CTAs instead, when that
+        // keeps the longest range as short (no range spans two row blocks, so a row block
+        // has fewer parts for the next level to read)
+        if (lv.U >= grid) {
+            const int64_t longest = (lv.U + grid - 1) / grid;
+            int64_t need = 0;
+            for (int ei = lv.e0; ei < lv.e0 + lv.ne; ++ei)
+                need += (int64_t)ent[ei].R * ((ent[ei].S + longest - 1) / longest);
+            if (need <= grid) {
+                int cc = 0;
+                for (int ei = lv.e0; ei < lv.e0 + lv.ne; ++ei) {
+                    const StackEntry &E = ent[ei];
+                    const int c_rb = (int)((E.S + longest - 1) / longest);  // CTAs per row block
+                    for (int rb = 0; rb < E.R; ++rb)
+                        for (int q = 0; q < c_rb; ++q)
+                            us[cc++] = (int)(E.unit_base + (int64_t)rb * E.S + (int64_t)E.S * q / c_rb);
+                }
+                for (; cc <= grid; ++cc) us[cc] = (int)lv.U;  // the CTAs left over have no tiles
+            }
+        }
         auto cta_of = [&](int64_t u) {  // the CTA whose range holds tile u
             return (int)(std::upper_bound(us, us + grid + 1, (int)u) - us) - 1;
         };
