@@ -36,9 +36,9 @@
 //     that have no slot to build while the others build (at the next start, before the
 //     build, if the next level reads that y directly). Those warps post their release as a
 //     ticket in shared memory; the producer warp takes it between two loads and makes the
-//     GPU-scope release, so no consumer waits for the rows' stores to land. A level waits for the sums of three
-//     levels back (the parts buffers rotate over three levels) and of every earlier level
-//     whose y it reads directly.
+//     GPU-scope release, so no consumer waits for the rows' stores to land. A level waits
+//     for the sums of three levels back (the parts buffers rotate over three levels) and
+//     of every earlier level whose y it reads directly.
 //   * Counters return to zero at the end of every launch (the last CTA to finish resets
 //     them), so the workspace can be replayed, e.g. from a CUDA graph.
 //
@@ -234,7 +234,6 @@ struct SlotSrc {
     const void *x;    // otherwise x itself
     int k0, K;        // first k of the stage; K of the GEMV
     int pm, st4;      // parts; their row stride in float4
-    int i;            // tile (relative to the CTA's first of the level)
 };
 
 // First scale group of k-stage s.
@@ -438,7 +437,6 @@ __global__ void __maxnreg__(128) gemv_stack(const StackArgs a) {
                 r.K = BE->K;
                 r.pm = BE->xpmax;
                 r.st4 = BE->xstride / 4;
-                r.i = i;
                 return r;
             };
             // the entry of level l - 2's block, read while the level waits
